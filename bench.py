@@ -1,0 +1,496 @@
+"""Device-timed benchmark of causal self-attention forward + backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one forward (gpt2_attn_fwd) plus one backward (the three steps of
+gpt2_attn_bwd) over one batch of the GPT-2 124M training shape B=16, T=1024,
+H=12, D=64, bf16 (seeded synthetic q, k, v, dO ~ N(0, 1)). The metric is
+causal attention fwd+bwd TFLOPS with the FLOPs counted as 2*B*H*T^2*D for the
+forward and 2.5x that for the backward, reported against the B200 dense bf16
+tensor-core peak.
+
+Timing: W untimed warm-up steps, then exactly K steps between CUDA events on
+the launching stream, with a barrier and torch.cuda.synchronize() on both
+sides; the max over ranks is taken. Each step uses the next of four input/
+output buffer sets (~0.8 GB in all), so no step finds its inputs in the
+126 MB L2. Events recorded between the four launches of every step give each
+kernel's average duration, which feeds the roofline object. With --gpus N > 1
+(torchrun, one process per GPU) every rank runs its own replica: attention
+has no exchange step, so the scaling is weak and there is no data-path
+collective.
+
+--impl reference times the CPU oracle (fp64 NumPy) on a bounded sample of the
+same workload on this host's cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "gpt2-124m-b16-t1024"
+METRIC = "causal attn fwd+bwd TFLOPS at GPT-2 124M shape (bf16), % of B200 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+N_SETS = 4
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def csrc_digest() -> str:
+    csrc = os.path.join(ROOT, "causal_self_attention_flashattention_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per launch from the last committed ncu capture, or {} when the
+    kernel sources changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    if d.get("csrc_digest") != csrc_digest():
+        return {}
+    return d.get("kernels", {})
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline and the --impl reference arm)
+# ---------------------------------------------------------------------------
+def _oracle_head(args):
+    Q, K, V, dO, scale = args
+    from oracle import oracle as orc
+
+    orc.head_forward(Q, K, V, scale)
+    orc.head_backward(Q, K, V, dO, scale)
+    return 0
+
+
+def _pool_init():
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
+
+
+class OracleTimer:
+    """Times the fp64 oracle's forward + backward on whole heads of the
+    workload, one head per worker process at a time."""
+
+    def __init__(self, wl, seed=0):
+        import multiprocessing as mp
+
+        from causal_self_attention_flashattention_b200.workload import make_inputs
+
+        self.wl = wl
+        self.cores = len(os.sched_getaffinity(0))
+        qkv, dout = make_inputs(1, wl.T, min(wl.H, 4), wl.D, seed=seed, qk_std=wl.qk_std)
+        q64 = qkv.double().numpy()
+        d64 = dout.double().numpy()
+        self.heads = [(q64[0, :, 0, h].copy(), q64[0, :, 1, h].copy(), q64[0, :, 2, h].copy(),
+                       d64[0, :, h].copy(), wl.scale) for h in range(q64.shape[3])]
+        self.pool = mp.get_context("spawn").Pool(self.cores, initializer=_pool_init)
+        self.pool.map(_oracle_head, [self.heads[0]] * self.cores)  # warm the workers
+
+    def head_flops(self):
+        wl = self.wl
+        return 7.0 * wl.T * wl.T * wl.D  # 2*T^2*D forward + 2.5x backward, one head
+
+    def run(self, n_heads):
+        tasks = [self.heads[i % len(self.heads)] for i in range(n_heads)]
+        t0 = time.perf_counter()
+        self.pool.map(_oracle_head, tasks, chunksize=1)
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    timer = OracleTimer(wl)
+    try:
+        n = timer.cores
+        elapsed = timer.run(n)
+        total_heads, total_t = n, elapsed
+        while total_t < budget_s:
+            n_more = max(timer.cores, int(timer.cores * (budget_s - total_t) / max(elapsed, 1e-3)))
+            n_more = min(n_more, 8 * timer.cores)
+            elapsed = timer.run(n_more)
+            total_heads += n_more
+            total_t += elapsed
+        tflops = total_heads * timer.head_flops() / total_t / 1e12
+        return {"value": tflops, "unit": "TFLOPS", "cores": timer.cores, "kind": "oracle",
+                "sample": f"{total_heads} whole heads (T={wl.T}, D={wl.D}) of {wl.name}, fp64 "
+                          f"NumPy fwd+bwd, one process per core, {total_t:.1f} s"}
+    finally:
+        timer.close()
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    timer = OracleTimer(wl)
+    try:
+        n = timer.cores
+        for _ in range(args.warmup):
+            timer.run(n)
+        t = 0.0
+        for _ in range(args.steps):
+            t += timer.run(n)
+        flops = args.steps * n * timer.head_flops()
+        value = flops / t / 1e12
+        line = {
+            "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "D": wl.D,
+                       "step": f"{n} whole heads of the workload (one per core)"},
+            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": timer.cores,
+                             "kind": "oracle",
+                             "sample": f"{n} heads (T={wl.T}, D={wl.D}) per step, fp64 NumPy "
+                                       "fwd+bwd, one process per core"},
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+    finally:
+        timer.close()
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# The CUDA path
+# ---------------------------------------------------------------------------
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+
+    # The oracle's worker pool (spawned) is started before any kernel runs.
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, budget_s=args.cpu_seconds)
+
+    from causal_self_attention_flashattention_b200 import build
+    build.build()
+    from causal_self_attention_flashattention_b200 import ops
+    from causal_self_attention_flashattention_b200.workload import (algorithmic_bytes,
+                                                                    attention_flops, make_inputs)
+
+    B, T, H, D, scale = wl.B, wl.T, wl.H, wl.D, wl.scale
+    qkv_cpu, dout_cpu = make_inputs(B, T, H, D, seed=rank, qk_std=wl.qk_std)
+    n_sets = args.sets
+    sets = []
+    for _ in range(n_sets):
+        sets.append(dict(
+            qkv=qkv_cpu.to(dev), dout=dout_cpu.to(dev),
+            out=torch.empty(B, T, H, D, dtype=torch.bfloat16, device=dev),
+            lse=torch.empty(B, H, T, dtype=torch.float32, device=dev),
+            delta=torch.empty(B, H, T, dtype=torch.float32, device=dev),
+            dqkv=torch.empty(B, T, 3, H, D, dtype=torch.bfloat16, device=dev)))
+    stream = torch.cuda.current_stream()
+
+    def step(s, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ops.attn_fwd(s["qkv"], scale, out=s["out"], lse=s["lse"], stream=stream)
+        ops.attn_bwd_steps(s["qkv"], s["out"], s["dout"], s["lse"], s["delta"], s["dqkv"], scale,
+                           stream=stream, events=None if ev is None else ev[1:])
+
+    for i in range(args.warmup):
+        step(sets[i % n_sets])
+    torch.cuda.synchronize()
+    st, word = ops.last_device_status()
+    if st != ops.GA_OK:
+        raise RuntimeError(f"device status after warm-up: {ops.status_string(st)} ({word:#x})")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = None
+    if rank == 0:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+        sampler.start()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    t_start.record(stream)
+    for i in range(K):
+        step(sets[i % n_sets], evs[i])
+    evs[-1][4].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    st, word = ops.last_device_status()
+    if st != ops.GA_OK:
+        raise RuntimeError(f"device status after timing: {ops.status_string(st)} ({word:#x})")
+
+    total_ms = t_start.elapsed_time(t_end)
+    names = ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"]
+    per = {n: 0.0 for n in names}
+    for ev in evs:
+        for k, n in enumerate(names):
+            per[n] += ev[k].elapsed_time(ev[k + 1])
+    per = {n: v / K for n, v in per.items()}
+
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    fwd_flops, bwd_flops = attention_flops(B, T, H, D)
+    step_flops = fwd_flops + bwd_flops
+    value = world * K * step_flops / (total_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak_tflops = float(peaks["bf16_tflops"])
+
+    # Per-kernel figures. Tensor-core kernels: the causal-triangle matmul FLOPs
+    # each one performs (units of B*H*T^2*D: fwd 2, dK/dV 4, dQ 3).
+    unit = float(B) * H * T * T * D
+    kflops = {"fwd": 2 * unit, "bwd_dkdv": 4 * unit, "bwd_dq": 3 * unit}
+    fwd_bytes, _ = algorithmic_bytes(B, T, H, D)
+    o_bytes = B * T * H * D * 2
+    lse_bytes = B * H * T * 4
+    qkv_bytes = 3 * o_bytes
+    kbytes = {
+        "fwd": fwd_bytes,
+        "bwd_preprocess": 2 * o_bytes + lse_bytes,
+        "bwd_dkdv": qkv_bytes + o_bytes + 2 * lse_bytes + 2 * o_bytes,
+        "bwd_dq": qkv_bytes + o_bytes + 2 * lse_bytes + o_bytes,
+    }
+    kernels = {}
+    for n in names:
+        ms = per[n]
+        d = {"ms": ms, "gbs": kbytes[n] / (ms * 1e-3) / 1e9}
+        if n in kflops:
+            d["tflops"] = kflops[n] / (ms * 1e-3) / 1e12
+            d["frac_of_peak"] = d["tflops"] / peak_tflops
+        else:
+            d["frac_of_hbm"] = d["gbs"] / float(peaks["hbm_gbs"])
+        kernels[n] = d
+    dominant = max(names, key=lambda n: per[n])
+    traffic = load_traffic()
+    dom = kernels[dominant]
+    if dominant in kflops:
+        roof = {"kernel": dominant, "bound": "tensor", "achieved": dom["tflops"],
+                "peak": peak_tflops, "unit": "TFLOP/s", "frac": dom["tflops"] / peak_tflops,
+                "peak_source": f"bf16_tflops (burst) of {peak_src}"}
+    else:
+        roof = {"kernel": dominant, "bound": "hbm", "achieved": dom["gbs"],
+                "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": dom["gbs"] / float(peaks["hbm_gbs"]), "peak_source": f"hbm_gbs of {peak_src}"}
+    roof["traffic"] = traffic.get(dominant, {}).get("dram_bytes_per_launch")
+
+    # End to end through the public API: pinned host buffers, copies in the timed region.
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wl, ops, dev, qkv_cpu, dout_cpu, step_flops, world)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "pct_of_peak": 100.0 * value / (world * peak_tflops),
+            "config": {"workload": wl.name, "B": B, "T": T, "H": H, "D": D, "scale": scale,
+                       "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
+                       "l2": f"{n_sets} rotating input/output sets "
+                             f"({n_sets * (2 * qkv_bytes + 3 * o_bytes) / 1e9:.2f} GB; "
+                             f"{2 * qkv_bytes + 3 * o_bytes + 2 * lse_bytes} B touched per step) "
+                             "> 126 MB L2",
+                       "step": "gpt2_attn_fwd + gpt2_attn_bwd (preprocess, dK/dV, dQ)"},
+            "clocks": clocks, "e2e": e2e, "gpu_launches": 4 * K,
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu,
+            "wall_s_timed_region": wall,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, wl, ops, dev, qkv_cpu, dout_cpu, step_flops, world):
+    import torch
+    import torch.distributed as dist
+
+    B, T, H, D, scale = wl.B, wl.T, wl.H, wl.D, wl.scale
+    h_qkv = qkv_cpu.pin_memory()
+    h_dout = dout_cpu.pin_memory()
+    h_out = torch.empty(B, T, H, D, dtype=torch.bfloat16).pin_memory()
+    h_lse = torch.empty(B, H, T, dtype=torch.float32).pin_memory()
+    h_dqkv = torch.empty(B, T, 3, H, D, dtype=torch.bfloat16).pin_memory()
+    d_qkv = torch.empty_like(qkv_cpu, device=dev)
+    d_dout = torch.empty_like(dout_cpu, device=dev)
+    d_out = torch.empty(B, T, H, D, dtype=torch.bfloat16, device=dev)
+    d_lse = torch.empty(B, H, T, dtype=torch.float32, device=dev)
+    d_dqkv = torch.empty(B, T, 3, H, D, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(ops.bwd_workspace_size(B, T, H, D), dtype=torch.uint8, device=dev)
+
+    def step():
+        d_qkv.copy_(h_qkv, non_blocking=True)
+        d_dout.copy_(h_dout, non_blocking=True)
+        ops.attn_fwd(d_qkv, scale, out=d_out, lse=d_lse)
+        ops.attn_bwd(d_qkv, d_out, d_dout, d_lse, scale, dqkv=d_dqkv, workspace=ws)
+        h_out.copy_(d_out, non_blocking=True)
+        h_lse.copy_(d_lse, non_blocking=True)
+        h_dqkv.copy_(d_dqkv, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    K = max(3, min(args.steps, args.e2e_steps))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(K):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = h_qkv.numel() * 2 + h_dout.numel() * 2
+    d2h = h_out.numel() * 2 + h_lse.numel() * 4 + h_dqkv.numel() * 2
+    return {"value": world * K * step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOPS",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+            "ms_per_step": ms / K}
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--e2e-steps", type=int, default=30)
+    p.add_argument("--sets", type=int, default=N_SETS,
+                   help="input/output buffer sets rotated through (default 4)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        p.error("--warmup must be at least 3")
+    from causal_self_attention_flashattention_b200.workload import WORKLOADS
+
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

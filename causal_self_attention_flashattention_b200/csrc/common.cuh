@@ -1,0 +1,44 @@
+// Shapes, tiling constants and the packed-QKV addressing shared by the
+// attention kernels.
+//
+// Packed QKV: element (b, t, s, h, d) of qkv (B, T, 3, H, D) sits at
+//     (((b*T + t)*3 + s)*H + h)*D + d,   s = 0 (q), 1 (k), 2 (v).
+// The TMA maps view it as a 3-D tensor {3*H*D, T, B} (innermost first), so the
+// 128-row tile of slot s, head h, rows [t0, t0+128) of batch b is the box at
+// coordinates {s*H*D + h*D, t0, b}. Rows past T read as zero.
+// out, dout (B, T, H, D) are viewed as {H*D, T, B} the same way.
+#pragma once
+
+#include <cstdint>
+
+namespace ga {
+
+constexpr int kD = 64;         // head dimension (GPT-2: 768 / 12)
+constexpr int kBlockM = 128;   // query rows per tile
+constexpr int kBlockN = 128;   // key rows per tile
+constexpr int kTileBytes = kBlockM * kD * 2;  // one 128 x 64 bf16 tile = 16 KiB
+
+// Wait-site codes reported in the device status word (high 32 bits).
+enum WaitSite : uint32_t {
+  kSiteFwdProducer = 0x101,
+  kSiteFwdMma = 0x102,
+  kSiteFwdSoftmax = 0x103,
+  kSiteFwdConvert = 0x104,
+  kFwdValueRange = 0x1F0,  // a V entry outside the fp16 range (|v| > 65504)
+  kSiteDqProducer = 0x201,
+  kSiteDqMma = 0x202,
+  kSiteDqSoftmax = 0x203,
+  kSiteDkvProducer = 0x301,
+  kSiteDkvMma = 0x302,
+  kSiteDkvSoftmax = 0x303,
+};
+
+struct AttnShape {
+  int B, T, H;
+  float scale_log2;   // scale * log2(e): logits in base-2 units
+  float scale;        // softmax scale (1/sqrt(D) for GPT-2)
+};
+
+__host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace ga

@@ -1,0 +1,422 @@
+// Forward kernel: out = softmax(scale * Q K^T + causal mask) V and the row
+// logsumexp, with the T x T matrix never leaving tensor memory / registers.
+//
+// Flash attention "never stores the full attention matrix" ("Let's reproduce
+// GPT-2 (124M)" video summary page, glossary table, row "flash attention").
+// This kernel does that as follows on sm_100a:
+//
+//   * Work item = one (batch, head) and a pair of adjacent 128-row query tiles
+//     (rows [256p, 256p+256)). Items run heaviest first over a persistent grid.
+//   * Warp 8 (TMA): loads the two Q tiles once per item (double-buffered
+//     across items) and streams the 128-row K and V tiles j = 0..2p+1 through a
+//     4-stage shared-memory ring.
+//   * Warp 9 (MMA, one thread): S_q = Q_q K_j^T (M128 N128 K64) into tensor
+//     memory, then O_q += P_q V_j (M128 N64 K128) with P_q read from tensor
+//     memory. Key tiles above the diagonal are never issued.
+//   * Warps 0-3 and 4-7 (softmax, one warpgroup per query tile, one row per
+//     thread): load the S row from tensor memory, apply the causal mask on the
+//     diagonal tile, run the online softmax in base 2 (running max m, running
+//     sum l), rescale O in tensor memory when m grows, and write P as fp16 back
+//     to tensor memory. At the end they normalise O, store out (bf16) and
+//     lse = ln2 * (m + log2 l).
+//   * Warps 10-11 (convert): rewrite each V tile in shared memory from bf16 to
+//     fp16 in place, so that O += P V runs as an fp16 x fp16 product. P in
+//     [0, 1] keeps 11 significant bits instead of 8, which matters on peaked
+//     rows where one probability near 1 multiplies a large v. Every bf16 value
+//     with |v| <= 65504 converts exactly (tiny ones to fp16 subnormals, within
+//     3e-8); a finite |v| above 65504 is reported in the status word.
+//
+// Tensor memory (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256),
+// P_0 [256,320), P_1 [320,384) (fp16 pairs), O_0 [384,448), O_1 [448,512).
+//
+// Registers: 384 threads launch with 168 each; the producer/MMA/convert
+// warpgroup drops to 88 and the two softmax warpgroups rise to 208
+// (128*88 + 256*208 = 384*168).
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace ga {
+namespace fwd {
+
+constexpr int kStages = 4;
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kConvertWarp0 = 10;  // warps 10 and 11
+// Register split (setmaxnreg): the producer/MMA/convert warpgroup gives up
+// registers to the two softmax warpgroups. The total must fit the block's
+// launch allocation (kThreads x kLaunchRegs), or setmaxnreg.inc would wait
+// forever; the host checks the compiled register count before any launch.
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kRegsAux = 88;
+constexpr uint32_t kRegsSoftmax = 208;
+static_assert(128 * kRegsAux + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+constexpr uint32_t kTmemCols = 512;
+
+__device__ __forceinline__ uint32_t col_s(int q) { return q * 128; }
+__device__ __forceinline__ uint32_t col_p(int q) { return 256 + q * 64; }
+__device__ __forceinline__ uint32_t col_o(int q) { return 384 + q * 64; }
+
+struct alignas(1024) Smem {
+  uint8_t q[2][2][kTileBytes];   // [item slot][query tile]
+  uint8_t k[kStages][kTileBytes];
+  uint8_t v[kStages][kTileBytes];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t kv_full[kStages], kv_empty[kStages], v_ready[kStages];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
+
+struct Item {
+  int b, h, i0, has1, n_kv;
+};
+
+__device__ __forceinline__ Item decode_item(int k, const AttnShape& sh) {
+  const int n_qt = ceil_div(sh.T, kBlockM);
+  const int n_pairs = ceil_div(n_qt, 2);
+  const int bh_count = sh.B * sh.H;
+  const int p = n_pairs - 1 - k / bh_count;  // heaviest pairs first
+  const int bh = k % bh_count;
+  Item it;
+  it.b = bh / sh.H;
+  it.h = bh % sh.H;
+  it.i0 = 2 * p;
+  it.has1 = (2 * p + 1) < n_qt;
+  it.n_kv = it.has1 ? 2 * p + 2 : 2 * p + 1;
+  return it;
+}
+
+__host__ __device__ __forceinline__ int num_items(const AttnShape& sh) {
+  return sh.B * sh.H * ceil_div(ceil_div(sh.T, kBlockM), 2);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __restrict__ out,
+                float* __restrict__ lse, const AttnShape sh) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                      ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int C = sh.H * kD;
+  const int n_items = num_items(sh);
+  volatile int* abort = &sm.abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.q_full[s], 1);
+      mbar_init(&sm.q_empty[s], 1);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.v_ready[s], 2);  // one arrival per convert warp
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&sm.s_full[q], 1);
+      mbar_init(&sm.s_free[q], 4);
+      mbar_init(&sm.p_full[q], 4);
+      mbar_init(&sm.o_done[q], 1);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kProducerWarp && lane == 0) tma_prefetch_desc(&map_qkv);
+  if (warp == kMmaWarp) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (warp >= kProducerWarp) {
+  regs_dealloc<kRegsAux>();
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ TMA warp
+    if (lane == 0) {
+      uint32_t kv_it = 0, it_cnt = 0;
+      for (int k = blockIdx.x; k < n_items; k += gridDim.x) {
+        const Item it = decode_item(k, sh);
+        const int slot = it_cnt & 1;
+        if (!mbar_wait(&sm.q_empty[slot], ((it_cnt >> 1) & 1) ^ 1, kSiteFwdProducer, abort)) break;
+        mbar_arrive_expect_tx(&sm.q_full[slot], (it.has1 ? 2 : 1) * kTileBytes);
+        tma_load_3d(sm.q[slot][0], &map_qkv, &sm.q_full[slot], it.h * kD, it.i0 * kBlockM, it.b);
+        if (it.has1)
+          tma_load_3d(sm.q[slot][1], &map_qkv, &sm.q_full[slot], it.h * kD,
+                      (it.i0 + 1) * kBlockM, it.b);
+        ++it_cnt;
+        bool ok = true;
+        for (int j = 0; j < it.n_kv; ++j, ++kv_it) {
+          const int s = kv_it % kStages;
+          if (!mbar_wait(&sm.kv_empty[s], ((kv_it / kStages) & 1) ^ 1, kSiteFwdProducer, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kTileBytes);
+          tma_load_3d(sm.k[s], &map_qkv, &sm.kv_full[s], C + it.h * kD, j * kBlockN, it.b);
+          tma_load_3d(sm.v[s], &map_qkv, &sm.kv_full[s], 2 * C + it.h * kD, j * kBlockN, it.b);
+        }
+        if (!ok) break;
+      }
+      // Drain: wait (bounded) for the last load issued into every buffer, so
+      // no copy is still landing in shared memory when the CTA exits.
+      for (int s = 0; s < kStages; ++s)
+        if (kv_it > static_cast<uint32_t>(s))
+          drain_wait(&sm.kv_full[s], ((kv_it - s + kStages - 1) / kStages - 1) & 1, kSiteFwdProducer);
+      for (int s = 0; s < 2; ++s)
+        if (it_cnt > static_cast<uint32_t>(s))
+          drain_wait(&sm.q_full[s], ((it_cnt - s + 1) / 2 - 1) & 1, kSiteFwdProducer);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA warp
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_o = idesc_f16_f32(128, 64, 0, 1);
+      uint32_t kv_it = 0, it_cnt = 0;
+      uint32_t s_cnt0 = 0, s_cnt1 = 0, p_cnt0 = 0, p_cnt1 = 0;
+      bool ok = true;
+      for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x, ++it_cnt) {
+        const Item it = decode_item(k, sh);
+        const int slot = it_cnt & 1;
+        if (!mbar_wait(&sm.q_full[slot], (it_cnt >> 1) & 1, kSiteFwdMma, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t qdesc0 = smem_desc_sw128(smem_u32(sm.q[slot][0]), 16, 1024);
+        const uint64_t qdesc1 = smem_desc_sw128(smem_u32(sm.q[slot][1]), 16, 1024);
+        for (int j = 0; j < it.n_kv; ++j, ++kv_it) {
+          const int s = kv_it % kStages;
+          if (!mbar_wait(&sm.kv_full[s], (kv_it / kStages) & 1, kSiteFwdMma, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t kdesc = smem_desc_sw128(smem_u32(sm.k[s]), 16, 1024);
+          const uint64_t vdesc = smem_desc_sw128(smem_u32(sm.v[s]), 128 * 128, 1024);
+          const bool active0 = j <= it.i0;
+          const bool active1 = it.has1 && j <= it.i0 + 1;
+          // S_q = Q_q K_j^T for both query tiles (K = 64 in steps of 16 = 32 bytes).
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const bool act = q == 0 ? active0 : active1;
+            if (ok && act) {
+              const uint32_t n = q == 0 ? s_cnt0 : s_cnt1;
+              if (n > 0 && !mbar_wait(&sm.s_free[q], (n - 1) & 1, kSiteFwdMma, abort)) ok = false;
+              if (ok) {
+                tc_fence_after();
+                const uint64_t qd = q == 0 ? qdesc0 : qdesc1;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                  mma_ss(tmem + col_s(q), qd + 2 * kk, kdesc + 2 * kk, idesc_s, kk > 0);
+                mma_commit(&sm.s_full[q]);
+                if (q == 0) ++s_cnt0; else ++s_cnt1;
+              }
+            }
+          }
+          if (ok && !mbar_wait(&sm.v_ready[s], (kv_it / kStages) & 1, kSiteFwdMma, abort)) ok = false;
+          // O_q += P_q V_j (16 keys = 8 TMEM columns of P, 2048 bytes of V per step).
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const bool act = q == 0 ? active0 : active1;
+            if (ok && act) {
+              const uint32_t n = q == 0 ? p_cnt0 : p_cnt1;
+              if (!mbar_wait(&sm.p_full[q], n & 1, kSiteFwdMma, abort)) ok = false;
+              if (ok) {
+                if (q == 0) ++p_cnt0; else ++p_cnt1;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kBlockN / 16; ++kk)
+                  mma_ts(tmem + col_o(q), tmem + col_p(q) + 8 * kk, vdesc + 128 * kk, idesc_o,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&sm.o_done[q]);
+              }
+            }
+          }
+          mma_commit(&sm.kv_empty[s]);
+          if (!ok) break;
+        }
+        if (ok) mma_commit(&sm.q_empty[slot]);
+      }
+      // Drain: every MMA this thread issued has finished before TMEM is freed.
+      mma_commit(&sm.drain);
+      drain_wait(&sm.drain, 0, kSiteFwdMma);
+    }
+    __syncwarp();
+  } else if (warp >= kConvertWarp0) {
+    // ------------------------------------------------------------ convert V
+    const int ct = threadIdx.x - kConvertWarp0 * 32;  // 0..63
+    uint32_t kv_it = 0;
+    bool ok = true;
+    for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+      const Item it = decode_item(k, sh);
+      for (int j = 0; j < it.n_kv; ++j, ++kv_it) {
+        const int s = kv_it % kStages;
+        ok = mbar_wait(&sm.kv_full[s], (kv_it / kStages) & 1, kSiteFwdConvert, abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        uint4* tile = reinterpret_cast<uint4*>(sm.v[s]);
+        bool bad = false;
+#pragma unroll 4
+        for (int c = ct; c < kTileBytes / 16; c += 64) {
+          uint4 w = tile[c];
+          uint32_t* u = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(u[e] << 16);
+            const float hi = __uint_as_float(u[e] & 0xFFFF0000u);
+            u[e] = pack_f16(lo, hi);
+            bad |= (fabsf(lo) > 65504.f && fabsf(lo) != INFINITY) ||
+                   (fabsf(hi) > 65504.f && fabsf(hi) != INFINITY);
+          }
+          tile[c] = w;
+        }
+        if (bad) record_failure(kFwdValueRange);
+        // Generic-proxy stores must be visible to the tensor core (async proxy).
+        fence_proxy_async_smem();
+        __syncwarp();
+        if ((ct & 31) == 0) mbar_arrive(&sm.v_ready[s]);
+      }
+    }
+  }
+  } else {
+    regs_alloc<kRegsSoftmax>();
+    // ------------------------------------------------------------ softmax
+    const int q = warp >> 2;                       // query tile of the pair
+    const int r = ((warp & 3) << 5) + lane;        // row within the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
+    const uint32_t t_s = tmem + lane_base + col_s(q);
+    const uint32_t t_p = tmem + lane_base + col_p(q);
+    const uint32_t t_o = tmem + lane_base + col_o(q);
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+      const Item it = decode_item(k, sh);
+      if (q == 1 && !it.has1) continue;
+      const int i = it.i0 + q;
+      const int row = i * kBlockM + r;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j <= i; ++j) {
+        ok = mbar_wait(&sm.s_full[q], s_cnt & 1, kSiteFwdSoftmax, abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        float x[128];
+        {
+          uint32_t u[128];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tmem_ld32(t_s + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(u + 32 * c));
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_free[q]);
+
+        float mx = -INFINITY;
+        if (j == i) {
+          const int lim = row - j * kBlockN;  // columns c > lim are future keys
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            x[c] = (c > lim) ? -INFINITY : x[c] * sh.scale_log2;
+            mx = fmaxf(mx, x[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            x[c] *= sh.scale_log2;
+            mx = fmaxf(mx, x[c]);
+          }
+        }
+        const float m_new = fmaxf(m, mx);
+        const float alpha = ex2(m - m_new);
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          x[c] = ex2(x[c] - m_new);
+          sum += x[c];
+        }
+        l = l * alpha + sum;
+        m = m_new;
+
+        if (j > 0) {
+          // O must hold P_{j-1} V_{j-1} before it is rescaled and P is reused.
+          ok = mbar_wait(&sm.o_done[q], o_cnt & 1, kSiteFwdSoftmax, abort);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ++o_cnt;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            uint32_t o[64];
+            tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(o));
+            tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(t_o, *reinterpret_cast<uint32_t(*)[32]>(o));
+            tmem_st32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+            tmem_wait_st();
+          }
+        }
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pk[e] = pack_f16(x[64 * c + 2 * e], x[64 * c + 2 * e + 1]);
+            tmem_st32(t_p + 32 * c, pk);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full[q]);
+      }
+      if (!ok) break;
+
+      // Epilogue: O / l -> out (bf16), lse in natural log.
+      ok = mbar_wait(&sm.o_done[q], o_cnt & 1, kSiteFwdSoftmax, abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++o_cnt;
+      tc_fence_after();
+      uint32_t o[64];
+      tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(o));
+      tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      if (row < sh.T) {
+        const float inv_l = 1.f / l;
+        uint4* dst = reinterpret_cast<uint4*>(
+            out + ((static_cast<size_t>(it.b) * sh.T + row) * sh.H + it.h) * kD);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 w;
+          w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+          w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+          w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+          w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+          dst[v] = w;
+        }
+        lse[(static_cast<size_t>(it.b) * sh.H + it.h) * sh.T + row] =
+            (m + lg2(l)) * 0.69314718055994531f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace fwd
+}  // namespace ga

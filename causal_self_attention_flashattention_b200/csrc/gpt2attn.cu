@@ -1,0 +1,282 @@
+// Host side of the library: argument checks, TMA tensor maps over the packed
+// layouts, launch configuration and the extern "C" entry points declared in
+// include/gpt2attn.h.
+//
+// Nothing here allocates device memory. The only process-wide state is a
+// per-device cache of the SM count and of the kernels' shared-memory opt-in,
+// guarded by a mutex, and the device status word the kernels write when a
+// bounded wait gives up.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "gpt2attn.h"
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "fwd.cuh"
+#include "bwd.cuh"
+
+namespace {
+
+using ga::kD;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Per-device set-up, once: SM count and the dynamic shared-memory opt-in of
+// every kernel. Returns nullptr on failure.
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& info = g_devices[dev];
+  if (info.ready) return &info;
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return nullptr;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if (cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return nullptr;
+  if (cudaFuncSetAttribute(ga::fwd::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::fwd::kSmemBytes)) != cudaSuccess)
+    return nullptr;
+  // The forward kernel redistributes registers between warpgroups; that only
+  // works if it launches with the register count the split was sized for.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel) != cudaSuccess ||
+      fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
+    return nullptr;
+  if (cudaFuncSetAttribute(ga::bwd::dkdv::attn_bwd_dkdv_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::bwd::dkdv::kSmemBytes)) != cudaSuccess)
+    return nullptr;
+  if (cudaFuncSetAttribute(ga::bwd::dq::attn_bwd_dq_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::bwd::dq::kSmemBytes)) != cudaSuccess)
+    return nullptr;
+  info.ready = true;
+  return &info;
+}
+
+// 3-D bf16 tensor map {inner, T, B} with a {64, 128, 1} box, 128-byte swizzle
+// and zero fill outside the tensor (rows past T read as 0).
+bool make_map(CUtensorMap* map, const void* base, uint64_t inner, int T, int B) {
+  const cuuint64_t dims[3] = {inner, static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[2] = {inner * 2, inner * 2 * static_cast<cuuint64_t>(T)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), static_cast<cuuint32_t>(ga::kBlockM), 1};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                              dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape and scale checks shared by every entry point.
+ga_status check_shape(int B, int T, int H, int D) {
+  if (B < 1 || T < 1 || H < 1 || D < 1) return GA_ERR_INVALID_ARG;
+  if (D != kD) return GA_ERR_UNSUPPORTED;
+  const long double elems = static_cast<long double>(B) * T * 3 * H * D;
+  if (elems >= 2147483648.0L) return GA_ERR_INVALID_ARG;
+  return GA_OK;
+}
+
+ga_status check_scale(float scale) {
+  if (!std::isfinite(scale) || !(scale > 0.f)) return GA_ERR_INVALID_ARG;
+  return GA_OK;
+}
+
+ga::AttnShape make_shape(int B, int T, int H, float scale) {
+  ga::AttnShape sh;
+  sh.B = B;
+  sh.T = T;
+  sh.H = H;
+  sh.scale = scale;
+  sh.scale_log2 = scale * 1.4426950408889634f;
+  return sh;
+}
+
+size_t delta_bytes(int B, int T, int H) {
+  const size_t n = static_cast<size_t>(B) * H * T * sizeof(float);
+  return (n + 255) & ~static_cast<size_t>(255);
+}
+
+int grid_for(int items, int num_sms) { return items < num_sms ? items : num_sms; }
+
+}  // namespace
+
+extern "C" {
+
+ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int D,
+                        float scale, gpt2attn_stream_t stream) {
+  if (qkv == nullptr || out == nullptr || lse == nullptr) return GA_ERR_INVALID_ARG;
+  ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if ((st = check_scale(scale)) != GA_OK) return st;
+  if (!aligned16(qkv) || !aligned16(out) || !aligned16(lse)) return GA_ERR_ALIGNMENT;
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GA_ERR_CUDA;
+
+  CUtensorMap map_qkv;
+  if (!make_map(&map_qkv, qkv, static_cast<uint64_t>(3) * H * kD, T, B)) return GA_ERR_CUDA;
+  const ga::AttnShape sh = make_shape(B, T, H, scale);
+  const int items = ga::fwd::num_items(sh);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ga::fwd::attn_fwd_kernel<<<grid_for(items, info->num_sms), ga::fwd::kThreads,
+                             ga::fwd::kSmemBytes, s>>>(
+      map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh);
+  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+}
+
+ga_status gpt2_attn_bwd_workspace_size(int B, int T, int H, int D, size_t* bytes) {
+  if (bytes == nullptr) return GA_ERR_INVALID_ARG;
+  const ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  *bytes = delta_bytes(B, T, H);
+  return GA_OK;
+}
+
+ga_status gpt2_attn_bwd_preprocess(const void* out, const void* dout, float* delta, int B,
+                                   int T, int H, int D, gpt2attn_stream_t stream) {
+  if (out == nullptr || dout == nullptr || delta == nullptr) return GA_ERR_INVALID_ARG;
+  const ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(delta)) return GA_ERR_ALIGNMENT;
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GA_ERR_CUDA;
+  const ga::AttnShape sh = make_shape(B, T, H, 1.f);
+  const long long rows = static_cast<long long>(B) * T * H;
+  const long long blocks_needed = (rows * 8 + 255) / 256;
+  const long long cap = 16LL * info->num_sms;
+  const int blocks = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
+  ga::bwd::attn_bwd_pre_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta, sh);
+  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+}
+
+namespace {
+
+// Shared checks and tensor maps of the two tensor-core backward steps.
+struct BwdLaunch {
+  CUtensorMap map_qkv, map_do;
+  ga::AttnShape sh;
+  int grid;
+};
+
+ga_status prepare_bwd(const void* qkv, const void* dout, const float* lse, const float* delta,
+                      void* dqkv, int B, int T, int H, int D, float scale, BwdLaunch* L) {
+  if (qkv == nullptr || dout == nullptr || lse == nullptr || delta == nullptr || dqkv == nullptr)
+    return GA_ERR_INVALID_ARG;
+  ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if ((st = check_scale(scale)) != GA_OK) return st;
+  if (!aligned16(qkv) || !aligned16(dout) || !aligned16(lse) || !aligned16(delta) ||
+      !aligned16(dqkv))
+    return GA_ERR_ALIGNMENT;
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GA_ERR_CUDA;
+  if (!make_map(&L->map_qkv, qkv, static_cast<uint64_t>(3) * H * kD, T, B)) return GA_ERR_CUDA;
+  if (!make_map(&L->map_do, dout, static_cast<uint64_t>(H) * kD, T, B)) return GA_ERR_CUDA;
+  L->sh = make_shape(B, T, H, scale);
+  L->grid = grid_for(B * H * ga::ceil_div(T, ga::kBlockM), info->num_sms);
+  return GA_OK;
+}
+
+}  // namespace
+
+ga_status gpt2_attn_bwd_dkdv(const void* qkv, const void* dout, const float* lse,
+                             const float* delta, void* dqkv, int B, int T, int H, int D,
+                             float scale, gpt2attn_stream_t stream) {
+  BwdLaunch L;
+  const ga_status st = prepare_bwd(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, &L);
+  if (st != GA_OK) return st;
+  ga::bwd::dkdv::attn_bwd_dkdv_kernel<<<L.grid, ga::bwd::kThreads, ga::bwd::dkdv::kSmemBytes,
+                                        reinterpret_cast<cudaStream_t>(stream)>>>(
+      L.map_qkv, L.map_do, lse, delta, static_cast<__nv_bfloat16*>(dqkv), L.sh);
+  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+}
+
+ga_status gpt2_attn_bwd_dq(const void* qkv, const void* dout, const float* lse,
+                           const float* delta, void* dqkv, int B, int T, int H, int D,
+                           float scale, gpt2attn_stream_t stream) {
+  BwdLaunch L;
+  const ga_status st = prepare_bwd(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, &L);
+  if (st != GA_OK) return st;
+  ga::bwd::dq::attn_bwd_dq_kernel<<<L.grid, ga::bwd::kThreads, ga::bwd::dq::kSmemBytes,
+                                    reinterpret_cast<cudaStream_t>(stream)>>>(
+      L.map_qkv, L.map_do, lse, delta, static_cast<__nv_bfloat16*>(dqkv), L.sh);
+  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+}
+
+ga_status gpt2_attn_bwd(const void* qkv, const void* out, const void* dout, const float* lse,
+                        void* dqkv, void* workspace, size_t workspace_bytes, int B, int T, int H,
+                        int D, float scale, gpt2attn_stream_t stream) {
+  if (qkv == nullptr || out == nullptr || dout == nullptr || lse == nullptr || dqkv == nullptr)
+    return GA_ERR_INVALID_ARG;
+  ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if ((st = check_scale(scale)) != GA_OK) return st;
+  if (workspace == nullptr || workspace_bytes < delta_bytes(B, T, H)) return GA_ERR_WORKSPACE;
+  if (!aligned16(qkv) || !aligned16(out) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dqkv) || !aligned16(workspace))
+    return GA_ERR_ALIGNMENT;
+  float* delta = static_cast<float*>(workspace);
+  if ((st = gpt2_attn_bwd_preprocess(out, dout, delta, B, T, H, D, stream)) != GA_OK) return st;
+  if ((st = gpt2_attn_bwd_dkdv(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream)) != GA_OK)
+    return st;
+  return gpt2_attn_bwd_dq(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
+}
+
+ga_status gpt2_attn_last_device_status(gpt2attn_stream_t stream, unsigned long long* detail) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GA_ERR_CUDA;
+  unsigned long long word = 0;
+  if (cudaMemcpyFromSymbol(&word, ga::g_device_status, sizeof(word)) != cudaSuccess)
+    return GA_ERR_CUDA;
+  if (word != 0) {
+    const unsigned long long zero = 0;
+    if (cudaMemcpyToSymbol(ga::g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+      return GA_ERR_CUDA;
+  }
+  if (detail != nullptr) *detail = word;
+  if (word == 0) return GA_OK;
+  return (word >> 32) == ga::kFwdValueRange ? GA_ERR_RANGE : GA_ERR_TIMEOUT;
+}
+
+const char* gpt2_attn_status_string(ga_status s) {
+  switch (s) {
+    case GA_OK: return "GA_OK";
+    case GA_ERR_INVALID_ARG: return "GA_ERR_INVALID_ARG: null pointer, bad size or bad scale";
+    case GA_ERR_UNSUPPORTED: return "GA_ERR_UNSUPPORTED: only head dimension D = 64 is implemented";
+    case GA_ERR_ALIGNMENT: return "GA_ERR_ALIGNMENT: every pointer must be 16-byte aligned";
+    case GA_ERR_WORKSPACE: return "GA_ERR_WORKSPACE: workspace missing or too small";
+    case GA_ERR_CUDA: return "GA_ERR_CUDA: a CUDA call failed";
+    case GA_ERR_TIMEOUT: return "GA_ERR_TIMEOUT: a device-side wait gave up";
+    case GA_ERR_RANGE: return "GA_ERR_RANGE: a v entry outside the fp16 range (|v| > 65504)";
+  }
+  return "unknown ga_status";
+}
+
+int gpt2_attn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,248 @@
+"""Python binding of libgpt2attn.so: argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels. This module
+checks tensor shapes, dtypes and devices, allocates outputs through PyTorch
+(which owns device memory and streams), and passes raw pointers and the
+current CUDA stream to the C ABI declared in include/gpt2attn.h. If the
+library is missing, importing this module raises ImportError: there is no
+fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libgpt2attn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with "
+        "`python -m causal_self_attention_flashattention_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+# Status codes of the C ABI.
+GA_OK = 0
+GA_ERR_INVALID_ARG = 1
+GA_ERR_UNSUPPORTED = 2
+GA_ERR_ALIGNMENT = 3
+GA_ERR_WORKSPACE = 4
+GA_ERR_CUDA = 5
+GA_ERR_TIMEOUT = 6
+GA_ERR_RANGE = 7
+
+EXPORTED_SYMBOLS = (
+    "gpt2_attn_fwd",
+    "gpt2_attn_bwd_workspace_size",
+    "gpt2_attn_bwd",
+    "gpt2_attn_bwd_preprocess",
+    "gpt2_attn_bwd_dkdv",
+    "gpt2_attn_bwd_dq",
+    "gpt2_attn_last_device_status",
+    "gpt2_attn_status_string",
+    "gpt2_attn_version",
+)
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+_lib.gpt2_attn_fwd.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_fwd.restype = _i
+_lib.gpt2_attn_bwd_workspace_size.argtypes = [_i, _i, _i, _i, ctypes.POINTER(ctypes.c_size_t)]
+_lib.gpt2_attn_bwd_workspace_size.restype = _i
+_lib.gpt2_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                               _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_bwd.restype = _i
+_lib.gpt2_attn_bwd_preprocess.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp]
+_lib.gpt2_attn_bwd_preprocess.restype = _i
+_lib.gpt2_attn_bwd_dkdv.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_bwd_dkdv.restype = _i
+_lib.gpt2_attn_bwd_dq.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_bwd_dq.restype = _i
+_lib.gpt2_attn_last_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
+_lib.gpt2_attn_last_device_status.restype = _i
+_lib.gpt2_attn_status_string.argtypes = [_i]
+_lib.gpt2_attn_status_string.restype = ctypes.c_char_p
+_lib.gpt2_attn_version.argtypes = []
+_lib.gpt2_attn_version.restype = _i
+
+
+class AttnError(RuntimeError):
+    """A non-zero status from the C ABI."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.gpt2_attn_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(_lib.gpt2_attn_version())
+
+
+def _check(status: int, where: str) -> None:
+    if status != GA_OK:
+        raise AttnError(status, where)
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _expect(t: torch.Tensor, name: str, shape, dtype) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _dims(qkv: torch.Tensor):
+    if qkv.dim() != 5 or qkv.shape[2] != 3:
+        raise ValueError(f"qkv must be (B, T, 3, H, D), got {tuple(qkv.shape)}")
+    B, T, _, H, D = qkv.shape
+    return int(B), int(T), int(H), int(D)
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / (D ** 0.5)
+
+
+def attn_fwd(qkv: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None,
+             lse: torch.Tensor | None = None, stream=None):
+    """Causal attention forward: returns (out (B,T,H,D) bf16, lse (B,H,T) fp32)."""
+    B, T, H, D = _dims(qkv)
+    _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
+    scale = default_scale(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=qkv.device)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=qkv.device)
+    _expect(out, "out", (B, T, H, D), torch.bfloat16)
+    _expect(lse, "lse", (B, H, T), torch.float32)
+    _check(_lib.gpt2_attn_fwd(qkv.data_ptr(), out.data_ptr(), lse.data_ptr(), B, T, H, D,
+                              scale, _stream_ptr(stream)), "gpt2_attn_fwd")
+    return out, lse
+
+
+def bwd_workspace_size(B: int, T: int, H: int, D: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.gpt2_attn_bwd_workspace_size(B, T, H, D, ctypes.byref(n)),
+           "gpt2_attn_bwd_workspace_size")
+    return int(n.value)
+
+
+def attn_bwd(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor,
+             scale: float | None = None, dqkv: torch.Tensor | None = None,
+             workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Causal attention backward: returns dqkv (B,T,3,H,D) bf16.
+
+    ``workspace`` (a uint8 CUDA tensor of at least ``bwd_workspace_size`` bytes)
+    is allocated here when not given; after the call its first B*H*T fp32
+    values hold Delta = rowsum(dout * out).
+    """
+    B, T, H, D = _dims(qkv)
+    _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
+    _expect(out, "out", (B, T, H, D), torch.bfloat16)
+    _expect(dout, "dout", (B, T, H, D), torch.bfloat16)
+    _expect(lse, "lse", (B, H, T), torch.float32)
+    scale = default_scale(D) if scale is None else float(scale)
+    if dqkv is None:
+        dqkv = torch.empty_like(qkv)
+    _expect(dqkv, "dqkv", (B, T, 3, H, D), torch.bfloat16)
+    need = bwd_workspace_size(B, T, H, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=qkv.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.gpt2_attn_bwd(qkv.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                              dqkv.data_ptr(), workspace.data_ptr(), ws_bytes, B, T, H, D,
+                              scale, _stream_ptr(stream)), "gpt2_attn_bwd")
+    return dqkv
+
+
+def attn_bwd_steps(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor,
+                   delta: torch.Tensor, dqkv: torch.Tensor, scale: float | None = None,
+                   stream=None, events=None) -> torch.Tensor:
+    """The backward as its three separate C-ABI steps (preprocess, dK/dV, dQ).
+
+    Same result as ``attn_bwd``. ``delta`` is a caller-owned fp32 (B,H,T)
+    tensor. If ``events`` (four CUDA events) is given, they are recorded on
+    the stream before, between and after the three launches, so each step can
+    be timed on the device.
+    """
+    B, T, H, D = _dims(qkv)
+    _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
+    _expect(out, "out", (B, T, H, D), torch.bfloat16)
+    _expect(dout, "dout", (B, T, H, D), torch.bfloat16)
+    _expect(lse, "lse", (B, H, T), torch.float32)
+    _expect(delta, "delta", (B, H, T), torch.float32)
+    _expect(dqkv, "dqkv", (B, T, 3, H, D), torch.bfloat16)
+    scale = default_scale(D) if scale is None else float(scale)
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    sp = _stream_ptr(stream)
+    if events is not None:
+        events[0].record(stream)
+    _check(_lib.gpt2_attn_bwd_preprocess(out.data_ptr(), dout.data_ptr(), delta.data_ptr(),
+                                         B, T, H, D, sp), "gpt2_attn_bwd_preprocess")
+    if events is not None:
+        events[1].record(stream)
+    _check(_lib.gpt2_attn_bwd_dkdv(qkv.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                                   delta.data_ptr(), dqkv.data_ptr(), B, T, H, D, scale, sp),
+           "gpt2_attn_bwd_dkdv")
+    if events is not None:
+        events[2].record(stream)
+    _check(_lib.gpt2_attn_bwd_dq(qkv.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                                 delta.data_ptr(), dqkv.data_ptr(), B, T, H, D, scale, sp),
+           "gpt2_attn_bwd_dq")
+    if events is not None:
+        events[3].record(stream)
+    return dqkv
+
+
+def last_device_status(stream=None) -> tuple[int, int]:
+    """Synchronises the stream; returns (status, raw status word) and clears it."""
+    word = ctypes.c_ulonglong(0)
+    st = _lib.gpt2_attn_last_device_status(_stream_ptr(stream), ctypes.byref(word))
+    return int(st), int(word.value)
+
+
+class CausalSelfAttention(torch.autograd.Function):
+    """Autograd wrapper: y = attention(qkv), with both passes in the library."""
+
+    @staticmethod
+    def forward(ctx, qkv, scale=None):
+        out, lse = attn_fwd(qkv, scale)
+        ctx.save_for_backward(qkv, out, lse)
+        ctx.scale = scale
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        qkv, out, lse = ctx.saved_tensors
+        return attn_bwd(qkv, out, dout.contiguous(), lse, ctx.scale), None
+
+
+def causal_self_attention(qkv: torch.Tensor, scale: float | None = None) -> torch.Tensor:
+    """One-call causal self-attention on packed qkv (B,T,3,H,D) -> (B,T,H,D)."""
+    return CausalSelfAttention.apply(qkv, scale)

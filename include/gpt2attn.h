@@ -1,0 +1,157 @@
+/*
+ * gpt2attn.h: C ABI of the fused causal self-attention library (sm_100a).
+ *
+ * The operation is the attention step of every GPT-2 (124M) block: causal
+ * multi-head self-attention on the packed q,k,v activations, computed the
+ * "flash attention" way, without ever storing the T x T attention matrix
+ * ("Let's reproduce GPT-2 (124M)" video summary page, glossary table, row
+ * "flash attention"; "Andrej Karpathy - Lets reproduce GPT 2 124M" video
+ * description, chapter 02:00:18 "flash attention"). The model is 12 layers of
+ * width C = 768 (video summary page, closing summary paragraph), i.e. H = 12
+ * heads of D = 64.
+ *
+ * Definition (per batch b, head h; i = query row, j = key row):
+ *     s_ij  = scale * q_i . k_j  for j <= i (key j visible iff j <= i)
+ *     lse_i = ln sum_{j<=i} exp(s_ij)
+ *     P_ij  = exp(s_ij - lse_i),   out_i = sum_j P_ij v_j
+ * and its gradients dq, dk, dv for an upstream gradient dout.
+ *
+ * Layouts (all row-major, contiguous, device memory):
+ *     qkv   bf16 (B, T, 3, H, D)  the GPT-2 c_attn output (B, T, 3C) split into
+ *                                 q (slot 0), k (slot 1), v (slot 2), head-major
+ *     out   bf16 (B, T, H, D)     = (B, T, C), ready for c_proj
+ *     lse   fp32 (B, H, T)        natural log of the scaled logits' sum of exp
+ *     dout  bf16 (B, T, H, D)
+ *     dqkv  bf16 (B, T, 3, H, D)  overwritten: slot 0 = dq, 1 = dk, 2 = dv
+ *
+ * Conventions:
+ *   - Only D == 64 is supported (GA_ERR_UNSUPPORTED otherwise).
+ *   - B, T, H >= 1; B*T*3*H*D must be below 2^31 elements.
+ *   - Every pointer must be non-null and 16-byte aligned.
+ *   - scale must be finite and > 0; GPT-2 uses 1/sqrt(D) = 0.125.
+ *   - The caller owns every buffer, including the backward workspace. The
+ *     library allocates nothing per call and keeps no state between calls,
+ *     apart from a device status word that records a timed-out wait.
+ *   - Calls only enqueue work on `stream` (the legacy default stream when
+ *     NULL). They never synchronise. Arguments are checked before anything is
+ *     launched: on any error nothing is launched and the status says why.
+ *   - Inputs and outputs must not overlap.
+ *   - No dropout, no attention bias, and no non-causal mode.
+ */
+#ifndef GPT2ATTN_H_
+#define GPT2ATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; declared here so that this header
+ * needs no CUDA header. */
+typedef struct CUstream_st* gpt2attn_stream_t;
+
+typedef enum {
+  GA_OK = 0,
+  GA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad scale, size overflow */
+  GA_ERR_UNSUPPORTED = 2, /* a shape the kernels do not implement (D != 64) */
+  GA_ERR_ALIGNMENT = 3,   /* a pointer that is not 16-byte aligned */
+  GA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the query result */
+  GA_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed */
+  GA_ERR_TIMEOUT = 6,     /* a device-side wait gave up (see gpt2_attn_last_device_status) */
+  GA_ERR_RANGE = 7        /* the forward met a finite v entry with |v| > 65504 (fp16 range) */
+} ga_status;
+
+/*
+ * Forward: out and lse from qkv.
+ *   qkv   [in]  bf16 (B,T,3,H,D), device
+ *   out   [out] bf16 (B,T,H,D), device, fully overwritten
+ *   lse   [out] fp32 (B,H,T), device, fully overwritten
+ * Steps on the device: tiles of 128 queries stream 128-key tiles of K and V
+ * through shared memory (TMA), S = Q K^T and O += P V run on the tensor cores
+ * with fp32 accumulators in tensor memory, the online softmax runs in
+ * registers, key tiles above the diagonal are skipped, and lse is written
+ * per query row. S = Q K^T multiplies bf16 operands. O += P V multiplies
+ * fp16 operands: P keeps 11 significant bits, and each bf16 v converts to
+ * fp16 exactly when |v| <= 65504. A finite |v| above that is reported as
+ * GA_ERR_RANGE by gpt2_attn_last_device_status; the outputs of that call are
+ * then undefined.
+ */
+ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse,
+                        int B, int T, int H, int D, float scale,
+                        gpt2attn_stream_t stream);
+
+/*
+ * Size in bytes of the workspace gpt2_attn_bwd needs for this shape.
+ * Layout of the workspace: Delta, fp32 (B,H,T), at offset 0, where
+ * Delta[b,h,t] = sum_d dout[b,t,h,d] * out[b,t,h,d]. After a gpt2_attn_bwd
+ * call it holds that call's Delta.
+ */
+ga_status gpt2_attn_bwd_workspace_size(int B, int T, int H, int D, size_t* bytes);
+
+/*
+ * Backward: dqkv from qkv, out, dout and lse (out and lse as written by
+ * gpt2_attn_fwd for the same qkv and scale).
+ *   qkv, out, dout, lse [in]
+ *   dqkv      [out] bf16 (B,T,3,H,D), fully overwritten (not accumulated)
+ *   workspace [scratch] device, >= gpt2_attn_bwd_workspace_size bytes,
+ *             16-byte aligned, owned by the caller, must not be shared by
+ *             calls that run concurrently
+ * Three launches on `stream`: Delta = rowsum(dout * out); dk and dv per key
+ * tile, which recompute P from lse; dq per query tile, which recomputes P and
+ * accumulates dq in tensor memory with no atomics. The result is bitwise
+ * deterministic.
+ */
+ga_status gpt2_attn_bwd(const void* qkv, const void* out, const void* dout,
+                        const float* lse, void* dqkv,
+                        void* workspace, size_t workspace_bytes,
+                        int B, int T, int H, int D, float scale,
+                        gpt2attn_stream_t stream);
+
+/*
+ * The three steps of gpt2_attn_bwd as separate calls, with the same argument
+ * conventions. gpt2_attn_bwd is exactly these three, in this order, on one
+ * stream. `delta` is fp32 (B,H,T), caller-owned, 16-byte aligned.
+ *
+ * gpt2_attn_bwd_preprocess: delta[b,h,t] = sum_d dout[b,t,h,d] * out[b,t,h,d]
+ *   (the row term sum_j P_ij dP_ij of the softmax Jacobian).
+ * gpt2_attn_bwd_dkdv: writes dqkv slots 1 (dk) and 2 (dv); slot 0 untouched.
+ *   One CTA per 128-key tile recomputes P from lse for every query tile at or
+ *   after it and accumulates dk, dv in tensor memory.
+ * gpt2_attn_bwd_dq: writes dqkv slot 0 (dq); slots 1 and 2 untouched. One CTA
+ *   per 128-query tile recomputes P and dP for every key tile at or before it
+ *   and accumulates dq in tensor memory (no atomics).
+ */
+ga_status gpt2_attn_bwd_preprocess(const void* out, const void* dout, float* delta,
+                                   int B, int T, int H, int D, gpt2attn_stream_t stream);
+ga_status gpt2_attn_bwd_dkdv(const void* qkv, const void* dout, const float* lse,
+                             const float* delta, void* dqkv,
+                             int B, int T, int H, int D, float scale,
+                             gpt2attn_stream_t stream);
+ga_status gpt2_attn_bwd_dq(const void* qkv, const void* dout, const float* lse,
+                           const float* delta, void* dqkv,
+                           int B, int T, int H, int D, float scale,
+                           gpt2attn_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word.
+ * Returns GA_ERR_TIMEOUT if a kernel of this library gave up on a device-side
+ * wait since the last call (the kernel then stopped early and its outputs are
+ * undefined), GA_ERR_RANGE if the forward met a v entry outside the fp16
+ * range, GA_ERR_CUDA if the synchronisation itself failed, GA_OK otherwise. If `detail` is non-null it receives the raw status word (0 when
+ * clean; otherwise the high 32 bits name the kernel and wait site and the
+ * low 32 bits the block index).
+ */
+ga_status gpt2_attn_last_device_status(gpt2attn_stream_t stream, unsigned long long* detail);
+
+/* Static, human-readable name of a status code. Never returns NULL. */
+const char* gpt2_attn_status_string(ga_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int gpt2_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPT2ATTN_H_ */

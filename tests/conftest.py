@@ -19,3 +19,11 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_sessionstart(session):
+    # The C-ABI library is built in-tree; (re)build it when missing or stale so
+    # that every test process loads the current sources.
+    from causal_self_attention_flashattention_b200 import build
+
+    build.build()

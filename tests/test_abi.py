@@ -1,0 +1,104 @@
+"""The C ABI: the library loads, exports every declared symbol, and rejects bad
+arguments with the documented status before anything reaches a device.
+
+Runs without a GPU: each call here fails argument checking, which happens
+before any CUDA call.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from causal_self_attention_flashattention_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+# A pointer value that is 16-byte aligned but never dereferenced (every call
+# below fails its checks first).
+P = 0x10000
+P_MIS = 0x10008
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)
+    return [n for n in names if n not in ("defined",)]
+
+
+def test_library_exports_every_declared_function():
+    decl = declared_functions()
+    assert "gpt2_attn_fwd" in decl and "gpt2_attn_bwd" in decl
+    for name in decl:
+        assert hasattr(ops.lib(), name), f"{name} declared in include/ but not exported"
+    assert set(ops.EXPORTED_SYMBOLS) <= set(decl)
+
+
+def test_status_strings_and_version():
+    for code in range(8):
+        s = ops.status_string(code)
+        assert s.startswith("GA_")
+    assert "unknown" in ops.status_string(99)
+    assert ops.version() >= 100
+
+
+def fwd(qkv=P, out=P, lse=P, B=1, T=128, H=12, D=64, scale=0.125):
+    return ops.lib().gpt2_attn_fwd(qkv, out, lse, B, T, H, D, scale, None)
+
+
+def bwd(qkv=P, out=P, dout=P, lse=P, dqkv=P, ws=P, ws_bytes=1 << 20,
+        B=1, T=128, H=12, D=64, scale=0.125):
+    return ops.lib().gpt2_attn_bwd(qkv, out, dout, lse, dqkv, ws, ws_bytes, B, T, H, D, scale, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(qkv=None), ops.GA_ERR_INVALID_ARG),
+    (dict(out=None), ops.GA_ERR_INVALID_ARG),
+    (dict(lse=None), ops.GA_ERR_INVALID_ARG),
+    (dict(B=0), ops.GA_ERR_INVALID_ARG),
+    (dict(T=-1), ops.GA_ERR_INVALID_ARG),
+    (dict(H=0), ops.GA_ERR_INVALID_ARG),
+    (dict(D=128), ops.GA_ERR_UNSUPPORTED),
+    (dict(D=32), ops.GA_ERR_UNSUPPORTED),
+    (dict(scale=0.0), ops.GA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), ops.GA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), ops.GA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), ops.GA_ERR_INVALID_ARG),
+    (dict(B=1 << 14, T=1 << 14, H=12), ops.GA_ERR_INVALID_ARG),  # >= 2^31 elements
+    (dict(qkv=P_MIS), ops.GA_ERR_ALIGNMENT),
+    (dict(out=P_MIS), ops.GA_ERR_ALIGNMENT),
+    (dict(lse=P + 4), ops.GA_ERR_ALIGNMENT),
+])
+def test_fwd_rejects(kw, status):
+    assert fwd(**kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dout=None), ops.GA_ERR_INVALID_ARG),
+    (dict(dqkv=None), ops.GA_ERR_INVALID_ARG),
+    (dict(D=80), ops.GA_ERR_UNSUPPORTED),
+    (dict(ws=None), ops.GA_ERR_WORKSPACE),
+    (dict(ws_bytes=16), ops.GA_ERR_WORKSPACE),
+    (dict(ws=P + 8), ops.GA_ERR_ALIGNMENT),
+    (dict(dqkv=P + 2), ops.GA_ERR_ALIGNMENT),
+    (dict(scale=0.0), ops.GA_ERR_INVALID_ARG),
+])
+def test_bwd_rejects(kw, status):
+    assert bwd(**kw) == status
+
+
+def test_workspace_size():
+    assert ops.bwd_workspace_size(16, 1024, 12, 64) == 16 * 12 * 1024 * 4
+    assert ops.bwd_workspace_size(1, 5, 1, 64) == 256  # rounded up to 256 bytes
+    n = ctypes.c_size_t(0)
+    assert ops.lib().gpt2_attn_bwd_workspace_size(1, 8, 1, 64, None) == ops.GA_ERR_INVALID_ARG
+    assert ops.lib().gpt2_attn_bwd_workspace_size(1, 8, 1, 48, ctypes.byref(n)) == ops.GA_ERR_UNSUPPORTED
+    with pytest.raises(ops.AttnError):
+        ops.bwd_workspace_size(0, 8, 1, 64)

@@ -1,0 +1,211 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle.
+
+Tolerances (on bf16-rounded inputs that both sides see):
+    out    max-abs error          <= 1e-2
+    lse    max-abs error          <= 1e-3
+    dq, dk, dv  relative Frobenius error  <= 2e-2 (per tensor)
+
+Small shapes compare every element. Shapes that span several tiles and a
+ragged tail (T not a multiple of 128) cover the tail handling. The five GPT-2
+workload shapes run the full problem on the GPU, in the same launch
+configuration the benchmark times, and compare sampled heads with the oracle
+computed head by head.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from causal_self_attention_flashattention_b200.workload import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 1e-2
+LSE_TOL = 1e-3
+GRAD_TOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def ops(cuda_device):
+    from causal_self_attention_flashattention_b200 import ops as _ops
+
+    return _ops
+
+
+def rel_fro(g, o):
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    den = np.linalg.norm(o)
+    return np.linalg.norm(g - o) / (den if den > 0 else 1.0)
+
+
+def run_gpu(ops, qkv_bf, dout_bf, scale):
+    qkv = qkv_bf.cuda()
+    dout = dout_bf.cuda()
+    out, lse = ops.attn_fwd(qkv, scale)
+    dqkv = ops.attn_bwd(qkv, out, dout, lse, scale)
+    st, word = ops.last_device_status()
+    assert st == ops.GA_OK, (st, hex(word))
+    return out.cpu(), lse.cpu(), dqkv.cpu()
+
+
+def check_all(ops, B, T, H, seed=0, qk_std=1.0, scale=0.125):
+    qkv_bf, dout_bf = make_inputs(B, T, H, 64, seed=seed, qk_std=qk_std)
+    out_g, lse_g, dqkv_g = run_gpu(ops, qkv_bf, dout_bf, scale)
+    out_o, lse_o, dqkv_o = orc.attention_forward_backward(
+        qkv_bf.double().numpy(), dout_bf.double().numpy(), scale,
+        processes=4 if B * H * T * T > 2**24 else None)
+    err_out = np.max(np.abs(out_g.double().numpy() - out_o))
+    err_lse = np.max(np.abs(lse_g.double().numpy() - lse_o))
+    g = dqkv_g.double().numpy()
+    errs = [rel_fro(g[:, :, s], dqkv_o[:, :, s]) for s in range(3)]
+    assert np.isfinite(g).all() and np.isfinite(out_g.double().numpy()).all()
+    assert err_out <= OUT_TOL, err_out
+    assert err_lse <= LSE_TOL, err_lse
+    assert max(errs) <= GRAD_TOL, errs
+    return err_out, err_lse, errs
+
+
+@pytest.mark.parametrize("B,T,H", [
+    (1, 128, 12),    # the small GPT-2 case: one tile per head
+    (1, 1, 1),       # a single token
+    (1, 8, 2),       # one partial tile
+    (2, 100, 3),     # ragged single tile
+    (1, 129, 2),     # one full tile + a 1-row tail
+    (2, 256, 2),     # exactly one query-tile pair
+    (1, 384, 3),     # odd number of tiles: the last pair has one tile
+    (1, 1000, 1),    # eight tiles, ragged
+    (3, 640, 2),     # five tiles
+])
+def test_fwd_bwd_matches_oracle(ops, B, T, H):
+    check_all(ops, B, T, H, seed=B * 1000 + T)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_small_gpt2_shape_seeds(ops, seed):
+    check_all(ops, 1, 128, 12, seed=seed)
+
+
+def test_peaked_softmax_rows(ops):
+    """q, k ~ N(0, 3^2): logits with std ~9 exercise the online rescale."""
+    check_all(ops, 1, 777, 2, seed=5, qk_std=3.0)
+
+
+def test_other_scale(ops):
+    check_all(ops, 1, 300, 2, seed=9, scale=0.05)
+
+
+def sampled_heads_check(ops, wl, heads, seed=0):
+    qkv_bf, dout_bf = make_inputs(wl.B, wl.T, wl.H, wl.D, seed=seed, qk_std=wl.qk_std)
+    out_g, lse_g, dqkv_g = run_gpu(ops, qkv_bf, dout_bf, wl.scale)
+    q64 = qkv_bf.double().numpy()
+    d64 = dout_bf.double().numpy()
+    for b, h in heads:
+        Q, K, V = (q64[b, :, s, h] for s in range(3))
+        O, lse, _ = orc.head_forward(Q, K, V, wl.scale)
+        dQ, dK, dV = orc.head_backward(Q, K, V, d64[b, :, h], wl.scale)
+        assert np.max(np.abs(out_g[b, :, h].double().numpy() - O)) <= OUT_TOL
+        assert np.max(np.abs(lse_g[b, h].double().numpy() - lse)) <= LSE_TOL
+        g = dqkv_g[b, :, :, h].double().numpy()
+        for s, ref in enumerate((dQ, dK, dV)):
+            assert rel_fro(g[:, s], ref) <= GRAD_TOL, (b, h, s, rel_fro(g[:, s], ref))
+    # Properties that hold at any size, over every head.
+    assert torch.isfinite(out_g.float()).all() and torch.isfinite(dqkv_g.float()).all()
+    # Query 0 attends only to key 0: out[:, 0] == v[:, 0] up to bf16 rounding.
+    assert torch.equal(out_g[:, 0], qkv_bf[:, 0, 2])
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("gpt2-124m-b16-t1024", [(0, 0), (7, 5), (15, 11)]),
+    ("gpt2-124m-b64-t1024", [(0, 3), (63, 11)]),
+    ("gpt2-350m-b32-t1024", [(1, 15), (31, 0)]),
+    ("stress-b4-t4096-qk3", [(0, 0), (3, 11)]),
+])
+def test_full_size_workloads_sampled_heads(ops, name, heads):
+    sampled_heads_check(ops, WORKLOADS[name], heads)
+
+
+def test_backward_is_deterministic(ops):
+    qkv_bf, dout_bf = make_inputs(2, 1024, 3, 64, seed=11)
+    qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
+    out, lse = ops.attn_fwd(qkv)
+    a = ops.attn_bwd(qkv, out, dout, lse)
+    b = ops.attn_bwd(qkv, out, dout, lse)
+    out2, lse2 = ops.attn_fwd(qkv)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+def test_outputs_written_exactly_in_bounds(ops):
+    """NaN-filled outputs inside canary padding: every output element is
+    written, and nothing outside the outputs changes."""
+    B, T, H, D = 2, 300, 3, 64
+    qkv_bf, dout_bf = make_inputs(B, T, H, D, seed=3)
+    qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
+    pad = 4096
+
+    def padded(shape, dtype, fill):
+        n = int(np.prod(shape))
+        buf = torch.full((n + 2 * pad,), 7.0, dtype=dtype, device="cuda")
+        view = buf[pad:pad + n].view(shape)
+        view.fill_(fill)
+        return buf, view
+
+    ob, out = padded((B, T, H, D), torch.bfloat16, float("nan"))
+    lb, lse = padded((B, H, T), torch.float32, float("nan"))
+    gb, dqkv = padded((B, T, 3, H, D), torch.bfloat16, float("nan"))
+    ws_need = ops.bwd_workspace_size(B, T, H, D)
+    wb, ws = padded((ws_need,), torch.uint8, 0)
+    ops.attn_fwd(qkv, out=out, lse=lse)
+    ops.attn_bwd(qkv, out, dout, lse, dqkv=dqkv, workspace=ws)
+    torch.cuda.synchronize()
+    for buf, view in ((ob, out), (lb, lse), (gb, dqkv)):
+        assert not torch.isnan(view).any()
+        assert (buf[:pad] == 7).all() and (buf[-pad:] == 7).all()
+    assert (wb[:pad] == 7).all() and (wb[-pad:] == 7).all()
+
+
+def test_delta_in_workspace(ops):
+    """The workspace holds Delta = rowsum(dout * out) after the backward."""
+    B, T, H, D = 2, 333, 3, 64
+    qkv_bf, dout_bf = make_inputs(B, T, H, D, seed=4)
+    qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
+    out, lse = ops.attn_fwd(qkv)
+    ws = torch.empty(ops.bwd_workspace_size(B, T, H, D), dtype=torch.uint8, device="cuda")
+    ops.attn_bwd(qkv, out, dout, lse, workspace=ws)
+    torch.cuda.synchronize()
+    delta_g = ws[: B * H * T * 4].view(torch.float32).view(B, H, T).cpu().double().numpy()
+    delta_o = orc.delta_rowsum(out.cpu().double().numpy(), dout_bf.double().numpy())
+    assert np.allclose(delta_g, delta_o, rtol=1e-5, atol=1e-5)
+
+
+def test_runs_on_a_side_stream(ops):
+    qkv_bf, dout_bf = make_inputs(1, 256, 2, 64, seed=6)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
+        out, lse = ops.attn_fwd(qkv)
+        dqkv = ops.attn_bwd(qkv, out, dout, lse)
+    s.synchronize()
+    out_o, lse_o, dqkv_o = orc.attention_forward_backward(
+        qkv_bf.double().numpy(), dout_bf.double().numpy(), 0.125)
+    assert np.max(np.abs(out.cpu().double().numpy() - out_o)) <= OUT_TOL
+    assert rel_fro(dqkv.cpu().double().numpy(), dqkv_o) <= GRAD_TOL
+
+
+def test_autograd_wrapper(ops):
+    qkv_bf, dout_bf = make_inputs(1, 200, 2, 64, seed=8)
+    x = qkv_bf.cuda().requires_grad_(True)
+    y = ops.causal_self_attention(x)
+    y.backward(dout_bf.cuda())
+    out_o, _, dqkv_o = orc.attention_forward_backward(
+        qkv_bf.double().numpy(), dout_bf.double().numpy(), 0.125)
+    assert np.max(np.abs(y.detach().cpu().double().numpy() - out_o)) <= OUT_TOL
+    assert rel_fro(x.grad.cpu().double().numpy(), dqkv_o) <= GRAD_TOL
+
+
+def test_status_word_clean_after_runs(ops):
+    st, word = ops.last_device_status()
+    assert st == ops.GA_OK and word == 0
