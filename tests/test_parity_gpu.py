@@ -1,7 +1,8 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle.
 
 Tolerances (on bf16-rounded inputs that both sides see):
-    out    max-abs error          <= 1e-2
+    out    max-abs error          <= 1e-2 (where the bf16 output grid allows it;
+                                   see out_error_ok)
     lse    max-abs error          <= 1e-3
     dq, dk, dv  relative Frobenius error  <= 2e-2 (per tensor)
 
@@ -24,6 +25,30 @@ pytestmark = pytest.mark.gpu
 OUT_TOL = 1e-2
 LSE_TOL = 1e-3
 GRAD_TOL = 2e-2
+
+
+def bf16_floor(o):
+    """|bf16(o) - o|: how far the nearest bf16 value lies from the exact output."""
+    o = np.asarray(o, dtype=np.float64)
+    return np.abs(torch.from_numpy(o).to(torch.bfloat16).double().numpy() - o)
+
+
+def out_error_ok(g, o):
+    """The out bound: max-abs error <= 1e-2 against the fp64 oracle.
+
+    out is bf16 by the library's layout. Where the exact value has no bf16
+    neighbour within 1e-2 (possible only for |o| >= 4, where the bf16 half-ulp
+    is 2^-6 = 0.0156), no bf16 output can meet the bound. There the element
+    passes only if it is no farther from the exact value than the correctly
+    rounded bf16 value is. Every other element must be within 1e-2.
+    Returns (ok, max error, number of elements at the bf16 floor).
+    """
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    err = np.abs(g - o)
+    floor = bf16_floor(o)
+    allowed = np.maximum(OUT_TOL, floor)
+    return bool(np.all(err <= allowed)), float(err.max()), int(np.sum(floor > OUT_TOL))
 
 
 @pytest.fixture(scope="module")
@@ -56,12 +81,12 @@ def check_all(ops, B, T, H, seed=0, qk_std=1.0, scale=0.125):
     out_o, lse_o, dqkv_o = orc.attention_forward_backward(
         qkv_bf.double().numpy(), dout_bf.double().numpy(), scale,
         processes=4 if B * H * T * T > 2**24 else None)
-    err_out = np.max(np.abs(out_g.double().numpy() - out_o))
+    ok_out, err_out, _ = out_error_ok(out_g.double().numpy(), out_o)
     err_lse = np.max(np.abs(lse_g.double().numpy() - lse_o))
     g = dqkv_g.double().numpy()
     errs = [rel_fro(g[:, :, s], dqkv_o[:, :, s]) for s in range(3)]
     assert np.isfinite(g).all() and np.isfinite(out_g.double().numpy()).all()
-    assert err_out <= OUT_TOL, err_out
+    assert ok_out, err_out
     assert err_lse <= LSE_TOL, err_lse
     assert max(errs) <= GRAD_TOL, errs
     return err_out, err_lse, errs
@@ -105,7 +130,8 @@ def sampled_heads_check(ops, wl, heads, seed=0):
         Q, K, V = (q64[b, :, s, h] for s in range(3))
         O, lse, _ = orc.head_forward(Q, K, V, wl.scale)
         dQ, dK, dV = orc.head_backward(Q, K, V, d64[b, :, h], wl.scale)
-        assert np.max(np.abs(out_g[b, :, h].double().numpy() - O)) <= OUT_TOL
+        ok_out, err_out, n_floor = out_error_ok(out_g[b, :, h].double().numpy(), O)
+        assert ok_out, (b, h, err_out, n_floor)
         assert np.max(np.abs(lse_g[b, h].double().numpy() - lse)) <= LSE_TOL
         g = dqkv_g[b, :, :, h].double().numpy()
         for s, ref in enumerate((dQ, dK, dV)):
@@ -191,7 +217,7 @@ def test_runs_on_a_side_stream(ops):
     s.synchronize()
     out_o, lse_o, dqkv_o = orc.attention_forward_backward(
         qkv_bf.double().numpy(), dout_bf.double().numpy(), 0.125)
-    assert np.max(np.abs(out.cpu().double().numpy() - out_o)) <= OUT_TOL
+    assert out_error_ok(out.cpu().double().numpy(), out_o)[0]
     assert rel_fro(dqkv.cpu().double().numpy(), dqkv_o) <= GRAD_TOL
 
 
@@ -202,7 +228,7 @@ def test_autograd_wrapper(ops):
     y.backward(dout_bf.cuda())
     out_o, _, dqkv_o = orc.attention_forward_backward(
         qkv_bf.double().numpy(), dout_bf.double().numpy(), 0.125)
-    assert np.max(np.abs(y.detach().cpu().double().numpy() - out_o)) <= OUT_TOL
+    assert out_error_ok(y.detach().cpu().double().numpy(), out_o)[0]
     assert rel_fro(x.grad.cpu().double().numpy(), dqkv_o) <= GRAD_TOL
 
 
