@@ -2,8 +2,9 @@
 
     python -m causal_self_attention_flashattention_b200.build [--verbose]
 
-The library is one CUDA translation unit (csrc/gpt2attn.cu, which includes the
-kernel headers) linked with the static CUDA runtime. It does not link against
+The library is built from the CUDA translation units in csrc/ (gpt2attn.cu,
+which includes the kernel headers, and noalloc.cu), linked with the static
+CUDA runtime. It does not link against
 libcuda: the tensor-map encoder is fetched at run time through
 cudaGetDriverEntryPoint. Cross-compiling needs no GPU.
 """
@@ -56,7 +57,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         _nvcc(), "-O3", "-std=c++17", *ARCH_FLAGS, "-lineinfo",
         "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
         f"-I{INCLUDE}", f"-I{CSRC}",
-        "-o", tmp, os.path.join(CSRC, "gpt2attn.cu"),
+        "-o", tmp, *[os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith(".cu")],
     ]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")

@@ -63,6 +63,8 @@ _lib.gpt2_attn_bwd_dkdv.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f,
 _lib.gpt2_attn_bwd_dkdv.restype = _i
 _lib.gpt2_attn_bwd_dq.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
 _lib.gpt2_attn_bwd_dq.restype = _i
+_lib.gpt2_attn_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_bwd_noalloc.restype = _i
 _lib.gpt2_attn_last_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
 _lib.gpt2_attn_last_device_status.restype = _i
 _lib.gpt2_attn_status_string.argtypes = [_i]
@@ -217,6 +219,31 @@ def attn_bwd_steps(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor, lse
            "gpt2_attn_bwd_dq")
     if events is not None:
         events[3].record(stream)
+    return dqkv
+
+
+def attn_bwd_noalloc(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+                     lse: torch.Tensor, scale: float | None = None, dqkv: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """The backward through gpt2_attn_bwd_noalloc: no workspace argument.
+
+    For callers that cannot allocate device memory; Delta lives in the
+    library's fixed static scratch (B*H*T <= 2^20), shared by all calls, so
+    calls that overlap on the GPU race. Pass a preallocated ``dqkv`` to make
+    the call itself allocate nothing.
+    """
+    B, T, H, D = _dims(qkv)
+    _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
+    _expect(out, "out", (B, T, H, D), torch.bfloat16)
+    _expect(dout, "dout", (B, T, H, D), torch.bfloat16)
+    _expect(lse, "lse", (B, H, T), torch.float32)
+    scale = default_scale(D) if scale is None else float(scale)
+    if dqkv is None:
+        dqkv = torch.empty_like(qkv)
+    _expect(dqkv, "dqkv", (B, T, 3, H, D), torch.bfloat16)
+    _check(_lib.gpt2_attn_bwd_noalloc(qkv.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                                      lse.data_ptr(), dqkv.data_ptr(), B, T, H, D, scale,
+                                      _stream_ptr(stream)), "gpt2_attn_bwd_noalloc")
     return dqkv
 
 

@@ -134,6 +134,32 @@ ga_status gpt2_attn_bwd_dq(const void* qkv, const void* dout, const float* lse,
                            gpt2attn_stream_t stream);
 
 /*
+ * gpt2_attn_bwd without a workspace argument, for callers that cannot
+ * allocate device memory: a plugin that is handed only its input and output
+ * buffers by a host application that owns all device memory, or a program
+ * that reserves the GPU's memory at start-up and may not call cudaMalloc (or
+ * pay for its implicit synchronisation) afterwards. The pages have no
+ * counterpart to this entry point; it exists for such callers only.
+ *   Same arguments, layouts and results as gpt2_attn_bwd. Delta is kept in a
+ *   fixed array in the library's static device memory instead of a caller
+ *   workspace: 2^20 floats (4 MiB) on every GPU that loads the library, held
+ *   until the process exits. Shapes with B*H*T > 1,048,576 are rejected with
+ *   GA_ERR_WORKSPACE before anything is launched.
+ *   Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   Every call shares the array and leaves its own Delta in it. Each call
+ *   rewrites all the Delta values it reads, so nothing needs clearing; but
+ *   calls that overlap on the GPU (other streams, other host threads on the
+ *   same device) race on the array and must be serialised by the caller.
+ */
+ga_status gpt2_attn_bwd_noalloc(const void* qkv, const void* out, const void* dout,
+                                const float* lse, void* dqkv,
+                                int B, int T, int H, int D, float scale,
+                                gpt2attn_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word.
  * Returns GA_ERR_TIMEOUT if a kernel of this library gave up on a device-side
  * wait since the last call (the kernel then stopped early and its outputs are
