@@ -66,9 +66,13 @@ attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* 
 }
 
 constexpr int kStages = 4;
-constexpr int kThreads = 192;  // warps 0-3 elementwise, 4 TMA, 5 MMA
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+// Warps 0-7: two elementwise warpgroups. Each thread owns one row of the tile
+// (its TMEM lane); warpgroup g takes the 64 columns [64g, 64g + 64).
+// Warp 8: TMA producer. Warp 9: MMA issuer.
+constexpr int kThreads = 320;
+constexpr int kEwWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -135,8 +139,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
       mbar_init(&sm.in_empty[s], 1);
     }
     mbar_init(&sm.sdp_full, 1);
-    mbar_init(&sm.sdp_free, 4);
-    mbar_init(&sm.ds_full, 4);
+    mbar_init(&sm.sdp_free, kEwWarps);
+    mbar_init(&sm.ds_full, kEwWarps);
     mbar_init(&sm.pds_free, 1);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -271,11 +275,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------- elementwise WG
-    const int r = (warp << 5) + lane;  // key row within the tile = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp << 5) << 16;
-    const uint32_t t_s = tmem + lane_base, t_dp = t_s + 128, t_p = t_s + 256, t_ds = t_s + 320;
-    const uint32_t t_dv = t_s + 384, t_dk = t_s + 448;
+    // ------------------------------------------------------- elementwise WGs
+    const int r = ((warp & 3) << 5) + lane;  // key row within the tile = TMEM lane
+    const int g = warp >> 2;                 // query columns [64g, 64g + 64)
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
+    const uint32_t t_s = tmem + lane_base + 64 * g, t_dp = tmem + lane_base + 128 + 64 * g;
+    const uint32_t t_p = tmem + lane_base + 256 + 32 * g, t_ds = tmem + lane_base + 320 + 32 * g;
+    const uint32_t t_dv = tmem + lane_base + 384 + 32 * g, t_dk = tmem + lane_base + 448 + 32 * g;
     uint32_t sdp_cnt = 0, pds_cnt = 0, in_it = 0;
     bool ok = true;
     for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
@@ -291,26 +297,24 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
         ++sdp_cnt;
         tc_fence_after();
         const bool diag = (i == j);
-        const float* l2 = sm.lse2[in_it % kStages];
-        const float* dl = sm.delta[in_it % kStages];
+        const float* l2 = sm.lse2[in_it % kStages] + 64 * g;
+        const float* dl = sm.delta[in_it % kStages] + 64 * g;
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sv[64], dv[64];
-          tmem_ld32(t_s + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(sv));
-          tmem_ld32(t_s + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-          tmem_ld32(t_dp + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(dv));
-          tmem_ld32(t_dp + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+        for (int half = 0; half < 2; ++half) {  // 32 query columns at a time
+          uint32_t sv[32], dv[32];
+          tmem_ld32(t_s + 32 * half, sv);
+          tmem_ld32(t_dp + 32 * half, dv);
           tmem_wait_ld();
           if (half == 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.sdp_free);
           }
-          uint32_t pp[32], dd[32];
+          uint32_t pp[16], dd[16];
 #pragma unroll
-          for (int c4 = 0; c4 < 16; ++c4) {
-            const float4 L = reinterpret_cast<const float4*>(l2 + 64 * half)[c4];
-            const float4 Dl = reinterpret_cast<const float4*>(dl + 64 * half)[c4];
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 L = reinterpret_cast<const float4*>(l2 + 32 * half)[c4];
+            const float4 Dl = reinterpret_cast<const float4*>(dl + 32 * half)[c4];
             const float lv[4] = {L.x, L.y, L.z, L.w};
             const float dlv[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
             float p[4], ds[4];
@@ -318,14 +322,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
             for (int e = 0; e < 4; ++e) {
               const int c = 4 * c4 + e;
               float x = fmaf(__uint_as_float(sv[c]), sh.scale_log2, -lv[e]);
-              if (diag && (64 * half + c) < r) x = -INFINITY;  // key r is after query c
+              if (diag && (64 * g + 32 * half + c) < r) x = -INFINITY;  // key r after query
               p[e] = ex2(x);
               ds[e] = p[e] * (__uint_as_float(dv[c]) - dlv[e]);
             }
-            pp[2 * c4] = pack_bf16(p[0], p[1]);
-            pp[2 * c4 + 1] = pack_bf16(p[2], p[3]);
-            dd[2 * c4] = pack_bf16(ds[0], ds[1]);
-            dd[2 * c4 + 1] = pack_bf16(ds[2], ds[3]);
+            pp[2 * c4] = pack_bf16_fast(p[0], p[1]);
+            pp[2 * c4 + 1] = pack_bf16_fast(p[2], p[3]);
+            dd[2 * c4] = pack_bf16_fast(ds[0], ds[1]);
+            dd[2 * c4 + 1] = pack_bf16_fast(ds[2], ds[3]);
           }
           if (half == 0 && i > j) {
             // The previous tile's dV/dK MMAs must be done reading P^T, dS^T.
@@ -335,8 +339,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
             ++pds_cnt;
             tc_fence_after();
           }
-          tmem_st32(t_p + 32 * half, pp);
-          tmem_st32(t_ds + 32 * half, dd);
+          tmem_st16(t_p + 16 * half, pp);
+          tmem_st16(t_ds + 16 * half, dd);
         }
         if (!ok) break;
         tmem_wait_st();
@@ -351,37 +355,30 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
       if (!ok) break;
       ++pds_cnt;
       tc_fence_after();
-      uint32_t a[64];
-      const int key = j * kBlockN + r;
-      __nv_bfloat16* base = dqkv + ((static_cast<size_t>(b) * sh.T + key) * 3) * C + h * kD;
-      // dV -> slot 2
-      tmem_ld32(t_dv, *reinterpret_cast<uint32_t(*)[32]>(a));
-      tmem_ld32(t_dv + 32, *reinterpret_cast<uint32_t(*)[32]>(a + 32));
-      tmem_wait_ld();
-      if (key < sh.T) {
-        uint4* dst = reinterpret_cast<uint4*>(base + 2 * C);
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = make_uint4(pack_bf16(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1])),
-                              pack_bf16(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3])),
-                              pack_bf16(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5])),
-                              pack_bf16(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7])));
-      }
-      // dK (times scale) -> slot 1
-      tmem_ld32(t_dk, *reinterpret_cast<uint32_t(*)[32]>(a));
-      tmem_ld32(t_dk + 32, *reinterpret_cast<uint32_t(*)[32]>(a + 32));
+      // Warpgroup g stores d columns [32g, 32g + 32) of dV and dK.
+      uint32_t av[32], ak[32];
+      tmem_ld32(t_dv, av);
+      tmem_ld32(t_dk, ak);
       tmem_wait_ld();
       tc_fence_before();
+      const int key = j * kBlockN + r;
       if (key < sh.T) {
+        __nv_bfloat16* base = dqkv + ((static_cast<size_t>(b) * sh.T + key) * 3) * C + h * kD + 32 * g;
+        uint4* dst_v = reinterpret_cast<uint4*>(base + 2 * C);
+        uint4* dst_k = reinterpret_cast<uint4*>(base + C);
         const float sc = sh.scale;
-        uint4* dst = reinterpret_cast<uint4*>(base + C);
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = make_uint4(
-              pack_bf16(__uint_as_float(a[8 * v]) * sc, __uint_as_float(a[8 * v + 1]) * sc),
-              pack_bf16(__uint_as_float(a[8 * v + 2]) * sc, __uint_as_float(a[8 * v + 3]) * sc),
-              pack_bf16(__uint_as_float(a[8 * v + 4]) * sc, __uint_as_float(a[8 * v + 5]) * sc),
-              pack_bf16(__uint_as_float(a[8 * v + 6]) * sc, __uint_as_float(a[8 * v + 7]) * sc));
+        for (int v = 0; v < 4; ++v) {
+          dst_v[v] = make_uint4(pack_bf16(__uint_as_float(av[8 * v]), __uint_as_float(av[8 * v + 1])),
+                                pack_bf16(__uint_as_float(av[8 * v + 2]), __uint_as_float(av[8 * v + 3])),
+                                pack_bf16(__uint_as_float(av[8 * v + 4]), __uint_as_float(av[8 * v + 5])),
+                                pack_bf16(__uint_as_float(av[8 * v + 6]), __uint_as_float(av[8 * v + 7])));
+          dst_k[v] = make_uint4(
+              pack_bf16(__uint_as_float(ak[8 * v]) * sc, __uint_as_float(ak[8 * v + 1]) * sc),
+              pack_bf16(__uint_as_float(ak[8 * v + 2]) * sc, __uint_as_float(ak[8 * v + 3]) * sc),
+              pack_bf16(__uint_as_float(ak[8 * v + 4]) * sc, __uint_as_float(ak[8 * v + 5]) * sc),
+              pack_bf16(__uint_as_float(ak[8 * v + 6]) * sc, __uint_as_float(ak[8 * v + 7]) * sc));
+        }
       }
     }
   }
@@ -456,8 +453,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
       mbar_init(&sm.kv_empty[s], 1);
     }
     mbar_init(&sm.sdp_full, 1);
-    mbar_init(&sm.sdp_free, 4);
-    mbar_init(&sm.ds_full, 4);
+    mbar_init(&sm.sdp_free, kEwWarps);
+    mbar_init(&sm.ds_full, kEwWarps);
     mbar_init(&sm.acc_done, 1);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -566,10 +563,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------- elementwise WG
-    const int r = (warp << 5) + lane;  // query row within the tile = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp << 5) << 16;
-    const uint32_t t_s = tmem + lane_base, t_dp = t_s + 128, t_ds0 = t_s + 256, t_dq = t_s + 384;
+    // ------------------------------------------------------- elementwise WGs
+    const int r = ((warp & 3) << 5) + lane;  // query row within the tile = TMEM lane
+    const int g = warp >> 2;                 // key columns [64g, 64g + 64)
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
+    const uint32_t t_s = tmem + lane_base + 64 * g, t_dp = tmem + lane_base + 128 + 64 * g;
+    const uint32_t t_ds0 = tmem + lane_base + 256 + 32 * g, t_dq = tmem + lane_base + 384 + 32 * g;
     uint32_t sdp_cnt = 0, acc_cnt = 0, ds_cnt = 0;
     bool ok = true;
     for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
@@ -589,35 +588,30 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
         const bool diag = (j == i);
         const uint32_t t_ds = t_ds0 + 64 * (ds_cnt & 1);
         ++ds_cnt;
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sv[64], dv[64];
-          tmem_ld32(t_s + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(sv));
-          tmem_ld32(t_s + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-          tmem_ld32(t_dp + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(dv));
-          tmem_ld32(t_dp + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
-          tmem_wait_ld();
-          if (half == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.sdp_free);
-          }
-          uint32_t dd[32];
+        uint32_t sv[64], dv[64];
+        tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sv));
+        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+        tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dv));
+        tmem_ld32(t_dp + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sdp_free);
+        uint32_t dd[32];
 #pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
-            float ds[2];
+        for (int c2 = 0; c2 < 32; ++c2) {
+          float ds[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int c = 2 * c2 + e;
-              float x = fmaf(__uint_as_float(sv[c]), sh.scale_log2, -lse2);
-              if (diag && (64 * half + c) > r) x = -INFINITY;  // key after query
-              const float p = ex2(x);
-              ds[e] = p * (__uint_as_float(dv[c]) - dlt);
-            }
-            dd[c2] = pack_bf16(ds[0], ds[1]);
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * c2 + e;
+            float x = fmaf(__uint_as_float(sv[c]), sh.scale_log2, -lse2);
+            if (diag && (64 * g + c) > r) x = -INFINITY;  // key after query
+            const float p = ex2(x);
+            ds[e] = p * (__uint_as_float(dv[c]) - dlt);
           }
-          tmem_st32(t_ds + 32 * half, dd);
+          dd[c2] = pack_bf16_fast(ds[0], ds[1]);
         }
+        tmem_st32(t_ds, dd);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -629,17 +623,17 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
       if (!ok) break;
       ++acc_cnt;
       tc_fence_after();
-      uint32_t a[64];
-      tmem_ld32(t_dq, *reinterpret_cast<uint32_t(*)[32]>(a));
-      tmem_ld32(t_dq + 32, *reinterpret_cast<uint32_t(*)[32]>(a + 32));
+      // Warpgroup g stores d columns [32g, 32g + 32) of dQ.
+      uint32_t a[32];
+      tmem_ld32(t_dq, a);
       tmem_wait_ld();
       tc_fence_before();
       if (valid) {
         const float sc = sh.scale;
         uint4* dst = reinterpret_cast<uint4*>(dqkv + ((static_cast<size_t>(b) * sh.T + row) * 3) * C +
-                                              h * kD);
+                                              h * kD + 32 * g);
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
+        for (int v = 0; v < 4; ++v)
           dst[v] = make_uint4(
               pack_bf16(__uint_as_float(a[8 * v]) * sc, __uint_as_float(a[8 * v + 1]) * sc),
               pack_bf16(__uint_as_float(a[8 * v + 2]) * sc, __uint_as_float(a[8 * v + 3]) * sc),

@@ -50,6 +50,9 @@ constexpr int kConvertWarp0 = 10;  // warps 10 and 11
 // launch allocation (kThreads x kLaunchRegs), or setmaxnreg.inc would wait
 // forever; the host checks the compiled register count before any launch.
 constexpr uint32_t kLaunchRegs = 168;
+// The running max is raised only when a row's max grows by more than this many
+// powers of two; until then P may reach 2^8 (well inside fp16).
+constexpr float kRescaleLog2 = 8.f;
 constexpr uint32_t kRegsAux = 88;
 constexpr uint32_t kRegsSoftmax = 208;
 static_assert(128 * kRegsAux + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
@@ -116,8 +119,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
-      mbar_init(&sm.v_ready[s], 2);  // one arrival per convert warp
+      mbar_init(&sm.kv_empty[s], 2);  // one arrival per query tile of the item
+      mbar_init(&sm.v_ready[s], 2);   // one arrival per convert warp
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(&sm.s_full[q], 1);
@@ -180,68 +183,92 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA warp
+    // Event-driven issue: the two query tiles of an item advance
+    // independently. Whenever a tile's next S product is possible (its key
+    // tile has landed and its softmax has read the previous S) or its next
+    // P V product is possible (P written, V converted), it is issued. One
+    // query tile therefore never waits on the other tile's softmax.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_o = idesc_f16_f32(128, 64, 0, 1);
       uint32_t kv_it = 0, it_cnt = 0;
-      uint32_t s_cnt0 = 0, s_cnt1 = 0, p_cnt0 = 0, p_cnt1 = 0;
+      uint32_t s_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
       bool ok = true;
       for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x, ++it_cnt) {
         const Item it = decode_item(k, sh);
         const int slot = it_cnt & 1;
         if (!mbar_wait(&sm.q_full[slot], (it_cnt >> 1) & 1, kSiteFwdMma, abort)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t qdesc0 = smem_desc_sw128(smem_u32(sm.q[slot][0]), 16, 1024);
-        const uint64_t qdesc1 = smem_desc_sw128(smem_u32(sm.q[slot][1]), 16, 1024);
-        for (int j = 0; j < it.n_kv; ++j, ++kv_it) {
-          const int s = kv_it % kStages;
-          if (!mbar_wait(&sm.kv_full[s], (kv_it / kStages) & 1, kSiteFwdMma, abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t kdesc = smem_desc_sw128(smem_u32(sm.k[s]), 16, 1024);
-          const uint64_t vdesc = smem_desc_sw128(smem_u32(sm.v[s]), 128 * 128, 1024);
-          const bool active0 = j <= it.i0;
-          const bool active1 = it.has1 && j <= it.i0 + 1;
-          // S_q = Q_q K_j^T for both query tiles (K = 64 in steps of 16 = 32 bytes).
+        const uint64_t qdesc[2] = {smem_desc_sw128(smem_u32(sm.q[slot][0]), 16, 1024),
+                                   smem_desc_sw128(smem_u32(sm.q[slot][1]), 16, 1024)};
+        // Key tiles seen by each query tile: 0..i0 and 0..i0+1 (if it exists).
+        const int n_tiles[2] = {it.i0 + 1, it.has1 ? it.i0 + 2 : 0};
+        int ns[2] = {0, 0}, np[2] = {0, 0};
+        // A stage is released by two arrivals, one per query tile. When only
+        // one query tile uses a key tile, issuing its P V product also makes
+        // the other tile's arrival (never earlier: an early arrival could
+        // complete the stage's previous phase).
+        uint64_t t_idle = 0;
+        while (np[0] < n_tiles[0] || np[1] < n_tiles[1]) {
+          bool progressed = false;
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
-            const bool act = q == 0 ? active0 : active1;
-            if (ok && act) {
-              const uint32_t n = q == 0 ? s_cnt0 : s_cnt1;
-              if (n > 0 && !mbar_wait(&sm.s_free[q], (n - 1) & 1, kSiteFwdMma, abort)) ok = false;
-              if (ok) {
+            // S_q(j) = Q_q K_j^T: needs K_j and the S_q buffer free.
+            if (ns[q] < n_tiles[q] && ns[q] <= np[q] + 1) {
+              const uint32_t idx = kv_it + ns[q];
+              const int st = idx % kStages;
+              if (mbar_test(&sm.kv_full[st], (idx / kStages) & 1) &&
+                  (s_cnt[q] == 0 || mbar_test(&sm.s_free[q], (s_cnt[q] - 1) & 1))) {
                 tc_fence_after();
-                const uint64_t qd = q == 0 ? qdesc0 : qdesc1;
+                const uint64_t kdesc = smem_desc_sw128(smem_u32(sm.k[st]), 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                  mma_ss(tmem + col_s(q), qd + 2 * kk, kdesc + 2 * kk, idesc_s, kk > 0);
+                for (int kk = 0; kk < kD / 16; ++kk)  // K = 64 in steps of 16 (32 bytes)
+                  mma_ss(tmem + col_s(q), qdesc[q] + 2 * kk, kdesc + 2 * kk, idesc_s, kk > 0);
                 mma_commit(&sm.s_full[q]);
-                if (q == 0) ++s_cnt0; else ++s_cnt1;
+                ++s_cnt[q];
+                ++ns[q];
+                progressed = true;
               }
             }
-          }
-          if (ok && !mbar_wait(&sm.v_ready[s], (kv_it / kStages) & 1, kSiteFwdMma, abort)) ok = false;
-          // O_q += P_q V_j (16 keys = 8 TMEM columns of P, 2048 bytes of V per step).
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const bool act = q == 0 ? active0 : active1;
-            if (ok && act) {
-              const uint32_t n = q == 0 ? p_cnt0 : p_cnt1;
-              if (!mbar_wait(&sm.p_full[q], n & 1, kSiteFwdMma, abort)) ok = false;
-              if (ok) {
-                if (q == 0) ++p_cnt0; else ++p_cnt1;
+            // O_q += P_q(j) V_j: needs P_q(j) written and V_j converted.
+            if (np[q] < ns[q]) {
+              const uint32_t idx = kv_it + np[q];
+              const int st = idx % kStages;
+              if (mbar_test(&sm.p_full[q], p_cnt[q] & 1) &&
+                  mbar_test(&sm.v_ready[st], (idx / kStages) & 1)) {
                 tc_fence_after();
+                const uint64_t vdesc = smem_desc_sw128(smem_u32(sm.v[st]), 128 * 128, 1024);
+                // 16 keys = 8 TMEM columns of P and 2048 bytes of V per step.
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk)
                   mma_ts(tmem + col_o(q), tmem + col_p(q) + 8 * kk, vdesc + 128 * kk, idesc_o,
-                         (j > 0 || kk > 0) ? 1u : 0u);
+                         (np[q] > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&sm.o_done[q]);
+                mma_commit(&sm.kv_empty[st]);
+                if (np[q] >= n_tiles[1 - q]) mbar_arrive(&sm.kv_empty[st]);
+                ++p_cnt[q];
+                ++np[q];
+                progressed = true;
               }
             }
           }
-          mma_commit(&sm.kv_empty[s]);
-          if (!ok) break;
+          if (progressed) {
+            t_idle = 0;
+          } else if (t_idle == 0) {
+            t_idle = globaltimer();
+          } else if (*abort) {
+            ok = false;
+            break;
+          } else if (globaltimer() - t_idle > kWaitTimeoutNs) {
+            record_failure(kSiteFwdMma);
+            *abort = 1;
+            ok = false;
+            break;
+          }
         }
-        if (ok) mma_commit(&sm.q_empty[slot]);
+        if (!ok) break;
+        kv_it += it.n_kv;
+        mma_commit(&sm.q_empty[slot]);
       }
       // Drain: every MMA this thread issued has finished before TMEM is freed.
       mma_commit(&sm.drain);
@@ -268,11 +295,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
           uint32_t* u = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float lo = __uint_as_float(u[e] << 16);
-            const float hi = __uint_as_float(u[e] & 0xFFFF0000u);
-            u[e] = pack_f16(lo, hi);
-            bad |= (fabsf(lo) > 65504.f && fabsf(lo) != INFINITY) ||
-                   (fabsf(hi) > 65504.f && fabsf(hi) != INFINITY);
+            bad |= bf16x2_out_of_f16_range(u[e]) != 0;
+            u[e] = bf16x2_to_f16x2(u[e]);
           }
           tile[c] = w;
         }
@@ -300,6 +324,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
       if (q == 1 && !it.has1) continue;
       const int i = it.i0 + q;
       const int row = i * kBlockM + r;
+      // Running max m (raw logit units, as read from S) and running sum l of
+      // 2^(s*c - m*c), c = scale*log2(e). m is only raised when the row max
+      // grows by more than kRescaleLog2 in log2 units; until then P and l keep
+      // using the stale m, which stays exact because O / l uses the same m.
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j <= i; ++j) {
         ok = mbar_wait(&sm.s_full[q], s_cnt & 1, kSiteFwdSoftmax, abort);
@@ -321,29 +349,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_free[q]);
 
-        float mx = -INFINITY;
         if (j == i) {
           const int lim = row - j * kBlockN;  // columns c > lim are future keys
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            x[c] = (c > lim) ? -INFINITY : x[c] * sh.scale_log2;
-            mx = fmaxf(mx, x[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            x[c] *= sh.scale_log2;
-            mx = fmaxf(mx, x[c]);
-          }
+          for (int c = 0; c < 128; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
         }
-        const float m_new = fmaxf(m, mx);
-        const float alpha = ex2(m - m_new);
-        float sum = 0.f;
+        // Row max: 8 independent chains of 3-input max.
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          x[c] = ex2(x[c] - m_new);
-          sum += x[c];
+        for (int e = 0; e < 8; ++e) mx8[e] = fmax3(x[e], x[8 + e], x[16 + e]);
+#pragma unroll
+        for (int c = 24; c < 128; c += 16) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], x[c + e], x[c + 8 + e]);
         }
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
+        const bool grow = (mx - m) * sh.scale_log2 > kRescaleLog2;  // always true on j == 0
+        const float m_new = grow ? mx : m;
+        const float alpha = grow ? ex2((m - m_new) * sh.scale_log2) : 1.f;
+        const float neg_mc = -m_new * sh.scale_log2;
+        // p = 2^(s*c - m*c), row sum, and fp16 packing of P in one pass, so the
+        // packing runs in the shadow of the exp2 calls.
+        uint32_t pk[64];
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c2 = 0; c2 < 64; ++c2) {
+          float y0, y1;
+          fma2(x[2 * c2], x[2 * c2 + 1], sh.scale_log2, neg_mc, y0, y1);
+          const float p0 = ex2(y0), p1 = ex2(y1);
+          add2(sa[c2 & 3], sb[c2 & 3], p0, p1);
+          pk[c2] = pack_f16_nonneg(p0, p1);
+        }
+        const float sum = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
         l = l * alpha + sum;
         m = m_new;
 
@@ -354,7 +392,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
           if (!ok) break;
           ++o_cnt;
           tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          if (__any_sync(0xffffffffu, grow)) {
             uint32_t o[64];
             tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(o));
             tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
@@ -366,16 +404,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
             tmem_wait_st();
           }
         }
-        {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) pk[e] = pack_f16(x[64 * c + 2 * e], x[64 * c + 2 * e + 1]);
-            tmem_st32(t_p + 32 * c, pk);
-          }
-          tmem_wait_st();
-        }
+        tmem_st32(t_p, *reinterpret_cast<uint32_t(*)[32]>(pk));
+        tmem_st32(t_p + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.p_full[q]);
@@ -407,7 +438,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
           dst[v] = w;
         }
         lse[(static_cast<size_t>(it.b) * sh.H + it.h) * sh.T + row] =
-            (m + lg2(l)) * 0.69314718055994531f;
+            (m * sh.scale_log2 + lg2(l)) * 0.69314718055994531f;
       }
     }
   }

@@ -75,6 +75,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   return ok != 0;
 }
 
+// Non-blocking check: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete. Returns false (after
 // recording `site`) on timeout, or when another role of the CTA has already
 // raised `*abort`.
@@ -291,6 +304,92 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ---------------------------------------------------------------------------
+// Float -> half conversions on the FMA/ALU pipes
+// ---------------------------------------------------------------------------
+// cvt.rn.{f16,bf16}x2.f32 runs on the same pipe as ex2.approx, which the
+// softmax keeps saturated. These equivalents use the FMA and integer pipes.
+
+// (a0 * s, a1 * s) in one packed fp32 multiply; round to nearest, subnormals
+// kept.
+__device__ __forceinline__ void mul2(float a0, float a1, float s, float& r0, float& r1) {
+  asm("{\n\t.reg .b64 a, b, r;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %4};\n\t"
+      "mul.rn.f32x2 r, a, b;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(s));
+}
+
+// (a0 * b + c, a1 * b + c) in one packed fp32 fused multiply-add.
+__device__ __forceinline__ void fma2(float a0, float a1, float b, float c, float& r0, float& r1) {
+  asm("{\n\t.reg .b64 a, b, c, r;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %4};\n\t"
+      "mov.b64 c, {%5, %5};\n\t"
+      "fma.rn.f32x2 r, a, b, c;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// (a0 + b0, a1 + b1) in one packed fp32 add.
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b;\n\t"
+      "mov.b64 a, {%0, %1};\n\t"
+      "mov.b64 b, {%2, %3};\n\t"
+      "add.rn.f32x2 a, a, b;\n\t"
+      "mov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// fp16 bits of a float x in [0, 65504]: x * 2^-112 moves the exponent bias
+// from 127 to 15, so bits [13, 29) of the product are the fp16 encoding,
+// subnormals included; +0x1000 rounds the 13 dropped bits (half up).
+constexpr float kF32ToF16Scale = 1.925929944387236e-34f;  // 2^-112
+
+__device__ __forceinline__ uint32_t pack_f16_nonneg(float lo, float hi) {
+  float m0, m1;
+  mul2(lo, hi, kF32ToF16Scale, m0, m1);
+  const uint32_t b0 = __float_as_uint(m0) + 0x1000u;
+  const uint32_t b1 = __float_as_uint(m1) + 0x1000u;
+  return (b0 >> 13) | ((b1 << 3) & 0xFFFF0000u);
+}
+
+// Two bf16 values (one 32-bit word) to two fp16 values. Exact for
+// |v| <= 65504 (subnormal results round half up); larger finite magnitudes
+// are not representable and must be caught with bf16x2_out_of_f16_range.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  float m0, m1;
+  mul2(__uint_as_float((w << 16) & 0x7FFF0000u), __uint_as_float(w & 0x7FFF0000u),
+       kF32ToF16Scale, m0, m1);
+  const uint32_t b0 = __float_as_uint(m0) + 0x1000u;
+  const uint32_t b1 = __float_as_uint(m1) + 0x1000u;
+  return (w & 0x80008000u) | (b0 >> 13) | ((b1 << 3) & 0x7FFF0000u);
+}
+
+// Nonzero iff a half of the bf16x2 word is finite with |v| >= 65536 (the
+// first bf16 magnitude above 65504).
+__device__ __forceinline__ uint32_t bf16x2_out_of_f16_range(uint32_t w) {
+  const uint32_t t = w & 0x7FFF7FFFu;
+  return ((t + 0x38803880u) & ~(t + 0x00800080u)) & 0x80008000u;
+}
+
+// Two floats to bf16x2, rounding half away from zero on the dropped bits
+// (differs from round-to-nearest-even only on exact ties).
+__device__ __forceinline__ uint32_t pack_bf16_fast(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 // Warpgroup-wide register budget changes (all four warps of a warpgroup
