@@ -66,13 +66,17 @@ attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* 
 }
 
 constexpr int kStages = 4;
-// Warps 0-7: two elementwise warpgroups. Each thread owns one row of the tile
-// (its TMEM lane); warpgroup g takes the 64 columns [64g, 64g + 64).
-// Warp 8: TMA producer. Warp 9: MMA issuer.
-constexpr int kThreads = 320;
-constexpr int kEwWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+// Warps 0-15: four elementwise warpgroups. Each thread owns one row of the
+// tile (its TMEM lane); warpgroup g takes the 32 columns [32g, 32g + 32).
+// Warp 16: TMA producer. Warp 17: issues the S and dP products (and owns the
+// tensor-memory allocation). Warp 18: issues the accumulating products (dV and
+// dK, or dQ). Two issuing threads let the next tile's S/dP enter the tensor
+// pipe while the current tile's accumulation waits for its elementwise step.
+constexpr int kThreads = 608;
+constexpr int kEwWarps = 16;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kAccWarp = 18;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -88,6 +92,100 @@ constexpr float kLog2e = 1.4426950408889634f;
 //   dK  += dS^T Q_i      (A = dS^T from tensor memory, B = Q_i MN-major)
 // Tensor memory: S^T [0,128), dP^T [128,256), P^T [256,320), dS^T [320,384)
 // (bf16 pairs), dV [384,448), dK [448,512).
+// 16 columns of one dK/dV tile row: P^T = 2^(S^T c - lse c) (zero where the
+// key r comes after query c0 + e when kMasked), dS^T = P^T (dP^T - Delta),
+// both packed to bf16 pairs.
+template <bool kMasked>
+__device__ __forceinline__ void dkdv_chunk(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
+                                           const float* nl, const float* nd, float sc, int c0,
+                                           int r, uint32_t (&pp)[8], uint32_t (&dd)[8]) {
+#pragma unroll
+  for (int e4 = 0; e4 < 4; ++e4) {
+    const float4 L = reinterpret_cast<const float4*>(nl)[e4];
+    const float4 Dl = reinterpret_cast<const float4*>(nd)[e4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = 4 * e4 + 2 * h;
+      float x0, x1, t0, t1, d0, d1;
+      fma2v(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sc, sc, h ? L.z : L.x,
+            h ? L.w : L.y, x0, x1);
+      if (kMasked) {
+        if (c0 + c < r) x0 = -INFINITY;
+        if (c0 + c + 1 < r) x1 = -INFINITY;
+      }
+      const float p0 = ex2(x0), p1 = ex2(x1);
+      t0 = __uint_as_float(dv[c]);
+      t1 = __uint_as_float(dv[c + 1]);
+      add2(t0, t1, h ? Dl.z : Dl.x, h ? Dl.w : Dl.y);
+      mul2v(p0, p1, t0, t1, d0, d1);
+      pp[c >> 1] = pack_bf16_fast(p0, p1);
+      dd[c >> 1] = pack_bf16_fast(d0, d1);
+    }
+  }
+}
+
+// 16 columns of one dQ tile row: P = 2^(S c - lse c) (zero where key
+// c0 + e comes after the query r when kMasked), dS = P (dP - Delta) as bf16
+// pairs. nl = -lse*log2(e) and nd = -Delta of the row.
+template <bool kMasked>
+__device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
+                                         float nl, float nd, float sc, int c0, int r,
+                                         uint32_t (&dd)[8]) {
+#pragma unroll
+  for (int c = 0; c < 16; c += 2) {
+    float x0, x1, d0, d1;
+    fma2v(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sc, sc, nl, nl, x0, x1);
+    if (kMasked) {
+      if (c0 + c > r) x0 = -INFINITY;
+      if (c0 + c + 1 > r) x1 = -INFINITY;
+    }
+    const float p0 = ex2(x0), p1 = ex2(x1);
+    float t0 = __uint_as_float(dv[c]), t1 = __uint_as_float(dv[c + 1]);
+    add2(t0, t1, nd, nd);
+    mul2v(p0, p1, t0, t1, d0, d1);
+    dd[c >> 1] = pack_bf16_fast(d0, d1);
+  }
+}
+
+// Stores one key row of dV (slot 2) and dK * scale (slot 1): warpgroup g
+// writes d columns [16g, 16g + 16) from its fp32 accumulator values.
+__device__ __forceinline__ void store_dkdv_row(__nv_bfloat16* dqkv, const uint32_t (&av)[16],
+                                               const uint32_t (&ak)[16], int b, int h, int j,
+                                               int r, int g, int C, const AttnShape& sh) {
+  const int key = j * kBlockN + r;
+  if (key >= sh.T) return;
+  __nv_bfloat16* base = dqkv + ((static_cast<size_t>(b) * sh.T + key) * 3) * C + h * kD + 16 * g;
+  uint4* dst_v = reinterpret_cast<uint4*>(base + 2 * C);
+  uint4* dst_k = reinterpret_cast<uint4*>(base + C);
+  const float s = sh.scale;
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    dst_v[v] = make_uint4(pack_bf16(__uint_as_float(av[8 * v]), __uint_as_float(av[8 * v + 1])),
+                          pack_bf16(__uint_as_float(av[8 * v + 2]), __uint_as_float(av[8 * v + 3])),
+                          pack_bf16(__uint_as_float(av[8 * v + 4]), __uint_as_float(av[8 * v + 5])),
+                          pack_bf16(__uint_as_float(av[8 * v + 6]), __uint_as_float(av[8 * v + 7])));
+    dst_k[v] = make_uint4(pack_bf16(__uint_as_float(ak[8 * v]) * s, __uint_as_float(ak[8 * v + 1]) * s),
+                          pack_bf16(__uint_as_float(ak[8 * v + 2]) * s, __uint_as_float(ak[8 * v + 3]) * s),
+                          pack_bf16(__uint_as_float(ak[8 * v + 4]) * s, __uint_as_float(ak[8 * v + 5]) * s),
+                          pack_bf16(__uint_as_float(ak[8 * v + 6]) * s, __uint_as_float(ak[8 * v + 7]) * s));
+  }
+}
+
+// Stores one query row of dQ * scale (slot 0), d columns [16g, 16g + 16).
+__device__ __forceinline__ void store_dq_row(__nv_bfloat16* dqkv, const uint32_t (&aq)[16], int b,
+                                             int h, int row, int g, int C, const AttnShape& sh) {
+  if (row >= sh.T) return;
+  const float s = sh.scale;
+  uint4* dst =
+      reinterpret_cast<uint4*>(dqkv + ((static_cast<size_t>(b) * sh.T + row) * 3) * C + h * kD + 16 * g);
+#pragma unroll
+  for (int v = 0; v < 2; ++v)
+    dst[v] = make_uint4(pack_bf16(__uint_as_float(aq[8 * v]) * s, __uint_as_float(aq[8 * v + 1]) * s),
+                        pack_bf16(__uint_as_float(aq[8 * v + 2]) * s, __uint_as_float(aq[8 * v + 3]) * s),
+                        pack_bf16(__uint_as_float(aq[8 * v + 4]) * s, __uint_as_float(aq[8 * v + 5]) * s),
+                        pack_bf16(__uint_as_float(aq[8 * v + 6]) * s, __uint_as_float(aq[8 * v + 7]) * s));
+}
+
 namespace dkdv {
 
 struct alignas(1024) Smem {
@@ -95,12 +193,12 @@ struct alignas(1024) Smem {
   uint8_t v[2][kTileBytes];
   uint8_t q[kStages][kTileBytes];
   uint8_t dout[kStages][kTileBytes];
-  float lse2[kStages][kBlockM];  // lse * log2(e) of the staged query tile
-  float delta[kStages][kBlockM];
+  float neg_lse2[kStages][kBlockM];  // -lse * log2(e) of the staged query tile
+  float neg_delta[kStages][kBlockM];  // -Delta of the staged query tile
   uint64_t kv_full[2], kv_empty[2];
   uint64_t in_full[kStages], in_empty[kStages];
   uint64_t sdp_full, sdp_free, ds_full, pds_free;
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -142,7 +240,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
     mbar_init(&sm.sdp_free, kEwWarps);
     mbar_init(&sm.ds_full, kEwWarps);
     mbar_init(&sm.pds_free, 1);
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain[0], 1);
+    mbar_init(&sm.drain[1], 1);
     sm.abort = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -165,7 +264,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
     // (base 2) and Delta values of each query tile next to its Q and dO tiles.
     uint32_t in_it = 0, it_cnt = 0;
     bool ok = true;
-    for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+    for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+      const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+      if (k >= n_items) continue;
       int b, h, j;
       decode(k, sh, b, h, j);
       const int slot = it_cnt & 1;
@@ -191,9 +292,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
           const int c = lane + 32 * e;
           const int qrow = i * kBlockM + c;
           const bool valid = qrow < sh.T;
-          // Rows past T get lse = +inf, so their P is exactly 0.
-          sm.lse2[s][c] = valid ? lse[row_base + qrow] * kLog2e : INFINITY;
-          sm.delta[s][c] = valid ? delta[row_base + qrow] : 0.f;
+          // Stored negated, so each becomes an addend of a fused multiply-add.
+          // Rows past T get -lse = -inf, so their P is exactly 0.
+          sm.neg_lse2[s][c] = valid ? -lse[row_base + qrow] * kLog2e : -INFINITY;
+          sm.neg_delta[s][c] = valid ? -delta[row_base + qrow] : 0.f;
         }
         __syncwarp();
         if (lane == 0) {
@@ -214,14 +316,15 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
+    // S^T = K_j Q_i^T and dP^T = V_j dO_i^T for every query tile i >= j.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, 64, 0, 1);
-      const uint32_t t_s = tmem + 0, t_dp = tmem + 128, t_p = tmem + 256, t_ds = tmem + 320;
-      const uint32_t t_dv = tmem + 384, t_dk = tmem + 448;
-      uint32_t in_it = 0, it_cnt = 0, sdp_cnt = 0, ds_cnt = 0;
+      const uint32_t t_s = tmem + 0, t_dp = tmem + 128;
+      uint32_t in_it = 0, it_cnt = 0, sdp_cnt = 0;
       bool ok = true;
-      for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x, ++it_cnt) {
+      for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+        const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+        if (k >= n_items) continue;
         int b, h, j;
         decode(k, sh, b, h, j);
         const int slot = it_cnt & 1;
@@ -230,61 +333,98 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
         const uint64_t kdesc = smem_desc_sw128(smem_u32(sm.k[slot]), 16, 1024);
         const uint64_t vdesc = smem_desc_sw128(smem_u32(sm.v[slot]), 16, 1024);
         const int n_i = n_qt - j;
-        // Issues S^T and dP^T for the idx-th query tile of this item.
-        auto issue_sdp = [&](uint32_t it_idx) -> bool {
-          const int s = it_idx % kStages;
-          if (!mbar_wait(&sm.in_full[s], (it_idx / kStages) & 1, kSiteDkvMma, abort)) return false;
-          if (sdp_cnt > 0 && !mbar_wait(&sm.sdp_free, (sdp_cnt - 1) & 1, kSiteDkvMma, abort))
-            return false;
+        for (int n = 0; n < n_i; ++n) {
+          const uint32_t idx = in_it + n;
+          const int s = idx % kStages;
+          if (!mbar_wait(&sm.in_full[s], (idx / kStages) & 1, kSiteDkvMma, abort)) { ok = false; break; }
+          if (sdp_cnt > 0 && !mbar_wait(&sm.sdp_free, (sdp_cnt - 1) & 1, kSiteDkvMma, abort)) { ok = false; break; }
           tc_fence_after();
           const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.q[s]), 16, 1024);
           const uint64_t odesc = smem_desc_sw128(smem_u32(sm.dout[s]), 16, 1024);
+          mma_ss(t_s, kdesc, qdesc, idesc_s, 0u);
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) mma_ss(t_s, kdesc + 2 * kk, qdesc + 2 * kk, idesc_s, kk > 0);
+          for (int kk = 1; kk < kD / 16; ++kk) mma_ss(t_s, kdesc + 2 * kk, qdesc + 2 * kk, idesc_s, 1u);
+          mma_ss(t_dp, vdesc, odesc, idesc_s, 0u);
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) mma_ss(t_dp, vdesc + 2 * kk, odesc + 2 * kk, idesc_s, kk > 0);
+          for (int kk = 1; kk < kD / 16; ++kk) mma_ss(t_dp, vdesc + 2 * kk, odesc + 2 * kk, idesc_s, 1u);
           mma_commit(&sm.sdp_full);
           ++sdp_cnt;
-          return true;
-        };
-        if (!issue_sdp(in_it)) { ok = false; break; }
+        }
+        if (!ok) break;
+        in_it += n_i;
+        ++it_cnt;
+      }
+      mma_commit(&sm.drain[0]);
+      drain_wait(&sm.drain[0], 0, kSiteDkvMma);
+    }
+    __syncwarp();
+  } else if (warp == kAccWarp) {
+    // dV += P^T dO_i and dK += dS^T Q_i once the elementwise step wrote them.
+    if (lane == 0) {
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, 64, 0, 1);
+      const uint32_t t_p = tmem + 256, t_ds = tmem + 320, t_dv = tmem + 384, t_dk = tmem + 448;
+      uint32_t in_it = 0, it_cnt = 0, ds_cnt = 0;
+      bool ok = true;
+      for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+        const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+        if (k >= n_items) continue;
+        int b, h, j;
+        decode(k, sh, b, h, j);
+        const int slot = it_cnt & 1;
+        const int n_i = n_qt - j;
         for (int n = 0; n < n_i; ++n) {
-          const uint32_t cur = in_it + n;
-          if (n + 1 < n_i && !issue_sdp(cur + 1)) { ok = false; break; }
+          const uint32_t idx = in_it + n;
+          const int s = idx % kStages;
+          // ds_full implies this stage's Q and dO landed and S^T/dP^T are done.
           if (!mbar_wait(&sm.ds_full, ds_cnt & 1, kSiteDkvMma, abort)) { ok = false; break; }
           ++ds_cnt;
           tc_fence_after();
-          const int s = cur % kStages;
           const uint64_t qdesc_mn = smem_desc_sw128(smem_u32(sm.q[s]), 128 * 128, 1024);
           const uint64_t odesc_mn = smem_desc_sw128(smem_u32(sm.dout[s]), 128 * 128, 1024);
+          const uint32_t acc0 = n > 0 ? 1u : 0u;
+          mma_ts(t_dv, t_p, odesc_mn, idesc_acc, acc0);
 #pragma unroll
-          for (int kk = 0; kk < kBlockM / 16; ++kk)
-            mma_ts(t_dv, t_p + 8 * kk, odesc_mn + 128 * kk, idesc_acc, (n > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 1; kk < kBlockM / 16; ++kk)
+            mma_ts(t_dv, t_p + 8 * kk, odesc_mn + 128 * kk, idesc_acc, 1u);
+          mma_ts(t_dk, t_ds, qdesc_mn, idesc_acc, acc0);
 #pragma unroll
-          for (int kk = 0; kk < kBlockM / 16; ++kk)
-            mma_ts(t_dk, t_ds + 8 * kk, qdesc_mn + 128 * kk, idesc_acc, (n > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 1; kk < kBlockM / 16; ++kk)
+            mma_ts(t_dk, t_ds + 8 * kk, qdesc_mn + 128 * kk, idesc_acc, 1u);
           mma_commit(&sm.pds_free);
           mma_commit(&sm.in_empty[s]);
         }
         if (!ok) break;
         in_it += n_i;
+        // Every S^T/dP^T of the item finished before its last dS^T was written,
+        // so this also releases K_j and V_j.
         mma_commit(&sm.kv_empty[slot]);
+        ++it_cnt;
       }
-      mma_commit(&sm.drain);
-      drain_wait(&sm.drain, 0, kSiteDkvMma);
+      mma_commit(&sm.drain[1]);
+      drain_wait(&sm.drain[1], 0, kSiteDkvMma);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------- elementwise WGs
     const int r = ((warp & 3) << 5) + lane;  // key row within the tile = TMEM lane
-    const int g = warp >> 2;                 // query columns [64g, 64g + 64)
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
-    const uint32_t t_s = tmem + lane_base + 64 * g, t_dp = tmem + lane_base + 128 + 64 * g;
-    const uint32_t t_p = tmem + lane_base + 256 + 32 * g, t_ds = tmem + lane_base + 320 + 32 * g;
-    const uint32_t t_dv = tmem + lane_base + 384 + 32 * g, t_dk = tmem + lane_base + 448 + 32 * g;
+    const int g = warp >> 2;                 // query columns [32g, 32g + 32)
+    const int r_lo = (warp & 3) << 5;        // first row of this warp
+    const uint32_t lb = static_cast<uint32_t>(r_lo) << 16;
+    const uint32_t t_s = tmem + lb + 32 * g, t_dp = tmem + lb + 128 + 32 * g;
+    const uint32_t t_p = tmem + lb + 256 + 16 * g, t_ds = tmem + lb + 320 + 16 * g;
+    const uint32_t t_dv = tmem + lb + 384 + 16 * g, t_dk = tmem + lb + 448 + 16 * g;
+    const float sc = sh.scale_log2;
     uint32_t sdp_cnt = 0, pds_cnt = 0, in_it = 0;
+    // The finished item whose dV, dK still sit in tensor memory: they are read
+    // out while the next item's first tile is processed, just before its P^T
+    // and dS^T go to tensor memory (after which the next dV/dK product
+    // overwrites the accumulators).
+    bool pending = false;
+    int pb = 0, ph = 0, pj = 0;
     bool ok = true;
-    for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+    for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+      const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+      if (k >= n_items) continue;
       int b, h, j;
       decode(k, sh, b, h, j);
       for (int i = j; i < n_qt; ++i, ++in_it) {
@@ -296,89 +436,85 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
         if (!ok) break;
         ++sdp_cnt;
         tc_fence_after();
-        const bool diag = (i == j);
-        const float* l2 = sm.lse2[in_it % kStages] + 64 * g;
-        const float* dl = sm.delta[in_it % kStages] + 64 * g;
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {  // 32 query columns at a time
-          uint32_t sv[32], dv[32];
-          tmem_ld32(t_s + 32 * half, sv);
-          tmem_ld32(t_dp + 32 * half, dv);
+        const float* nl = sm.neg_lse2[in_it % kStages] + 32 * g;
+        const float* nd = sm.neg_delta[in_it % kStages] + 32 * g;
+        // Both 16-column halves are computed into registers before waiting for
+        // the previous dV/dK products to release P^T and dS^T, so that wait
+        // overlaps all of this tile's elementwise work.
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sv[16], dv[16];
+          tmem_ld16(t_s + 16 * half, sv);
+          tmem_ld16(t_dp + 16 * half, dv);
           tmem_wait_ld();
           if (half == 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.sdp_free);
           }
-          uint32_t pp[16], dd[16];
-#pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 L = reinterpret_cast<const float4*>(l2 + 32 * half)[c4];
-            const float4 Dl = reinterpret_cast<const float4*>(dl + 32 * half)[c4];
-            const float lv[4] = {L.x, L.y, L.z, L.w};
-            const float dlv[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
-            float p[4], ds[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 4 * c4 + e;
-              float x = fmaf(__uint_as_float(sv[c]), sh.scale_log2, -lv[e]);
-              if (diag && (64 * g + 32 * half + c) < r) x = -INFINITY;  // key r after query
-              p[e] = ex2(x);
-              ds[e] = p[e] * (__uint_as_float(dv[c]) - dlv[e]);
-            }
-            pp[2 * c4] = pack_bf16_fast(p[0], p[1]);
-            pp[2 * c4 + 1] = pack_bf16_fast(p[2], p[3]);
-            dd[2 * c4] = pack_bf16_fast(ds[0], ds[1]);
-            dd[2 * c4 + 1] = pack_bf16_fast(ds[2], ds[3]);
-          }
-          if (half == 0 && i > j) {
-            // The previous tile's dV/dK MMAs must be done reading P^T, dS^T.
-            ok = mbar_wait(&sm.pds_free, pds_cnt & 1, kSiteDkvSoftmax, abort);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            ++pds_cnt;
-            tc_fence_after();
-          }
-          tmem_st16(t_p + 16 * half, pp);
-          tmem_st16(t_ds + 16 * half, dd);
+          const int c0 = 32 * g + 16 * half;  // first query column of the chunk
+          uint32_t (&pph)[8] = *reinterpret_cast<uint32_t(*)[8]>(pp + 8 * half);
+          uint32_t (&ddh)[8] = *reinterpret_cast<uint32_t(*)[8]>(dd + 8 * half);
+          // On the diagonal tile, a chunk needs the mask if one of its columns
+          // lies before one of this warp's rows (key after query).
+          if (i == j && c0 < r_lo + 31)
+            dkdv_chunk<true>(sv, dv, nl + 16 * half, nd + 16 * half, sc, c0, r, pph, ddh);
+          else
+            dkdv_chunk<false>(sv, dv, nl + 16 * half, nd + 16 * half, sc, c0, r, pph, ddh);
         }
-        if (!ok) break;
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.ds_full);
+        const bool flush = (i == j) && pending;
+        if (i > j || flush) {
+          // The previous dV/dK products must be done reading P^T and dS^T; on
+          // an item's first tile that is the finished item's last product.
+          ok = mbar_wait(&sm.pds_free, pds_cnt & 1, kSiteDkvSoftmax, abort);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ++pds_cnt;
+          tc_fence_after();
+        }
+        if (flush) {
+          // Read the finished item's accumulators out before this tile's dV/dK
+          // product overwrites them; store them once this tile is handed over.
+          uint32_t av[16], ak[16];
+          tmem_ld16(t_dv, av);
+          tmem_ld16(t_dk, ak);
+          tmem_wait_ld();
+          tmem_st16(t_p, pp);
+          tmem_st16(t_ds, dd);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.ds_full);
+          store_dkdv_row(dqkv, av, ak, pb, ph, pj, r, g, C, sh);
+          pending = false;
+        } else {
+          tmem_st16(t_p, pp);
+          tmem_st16(t_ds, dd);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.ds_full);
+        }
       }
       if (!ok) break;
-      // The last tile's pds_free phase: dV and dK are complete.
+      pending = true;
+      pb = b;
+      ph = h;
+      pj = j;
+    }
+    if (ok && pending) {
       ok = mbar_wait(&sm.pds_free, pds_cnt & 1, kSiteDkvSoftmax, abort);
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      ++pds_cnt;
-      tc_fence_after();
-      // Warpgroup g stores d columns [32g, 32g + 32) of dV and dK.
-      uint32_t av[32], ak[32];
-      tmem_ld32(t_dv, av);
-      tmem_ld32(t_dk, ak);
-      tmem_wait_ld();
-      tc_fence_before();
-      const int key = j * kBlockN + r;
-      if (key < sh.T) {
-        __nv_bfloat16* base = dqkv + ((static_cast<size_t>(b) * sh.T + key) * 3) * C + h * kD + 32 * g;
-        uint4* dst_v = reinterpret_cast<uint4*>(base + 2 * C);
-        uint4* dst_k = reinterpret_cast<uint4*>(base + C);
-        const float sc = sh.scale;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          dst_v[v] = make_uint4(pack_bf16(__uint_as_float(av[8 * v]), __uint_as_float(av[8 * v + 1])),
-                                pack_bf16(__uint_as_float(av[8 * v + 2]), __uint_as_float(av[8 * v + 3])),
-                                pack_bf16(__uint_as_float(av[8 * v + 4]), __uint_as_float(av[8 * v + 5])),
-                                pack_bf16(__uint_as_float(av[8 * v + 6]), __uint_as_float(av[8 * v + 7])));
-          dst_k[v] = make_uint4(
-              pack_bf16(__uint_as_float(ak[8 * v]) * sc, __uint_as_float(ak[8 * v + 1]) * sc),
-              pack_bf16(__uint_as_float(ak[8 * v + 2]) * sc, __uint_as_float(ak[8 * v + 3]) * sc),
-              pack_bf16(__uint_as_float(ak[8 * v + 4]) * sc, __uint_as_float(ak[8 * v + 5]) * sc),
-              pack_bf16(__uint_as_float(ak[8 * v + 6]) * sc, __uint_as_float(ak[8 * v + 7]) * sc));
-        }
+      if (ok) {
+        ++pds_cnt;
+        tc_fence_after();
+        uint32_t av[16], ak[16];
+        tmem_ld16(t_dv, av);
+        tmem_ld16(t_dk, ak);
+        tmem_wait_ld();
+        tc_fence_before();
+        store_dkdv_row(dqkv, av, ak, pb, ph, pj, r, g, C, sh);
       }
     }
   }
@@ -413,7 +549,8 @@ struct alignas(1024) Smem {
   uint64_t in_full[2], in_empty[2];
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t sdp_full, sdp_free, ds_full, acc_done;
-  uint64_t drain;
+  uint64_t ds_free[2];  // dS buffer b no longer read by a dQ product
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -456,7 +593,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
     mbar_init(&sm.sdp_free, kEwWarps);
     mbar_init(&sm.ds_full, kEwWarps);
     mbar_init(&sm.acc_done, 1);
-    mbar_init(&sm.drain, 1);
+    for (int d = 0; d < 2; ++d) {
+      mbar_init(&sm.ds_free[d], 1);
+      mbar_init(&sm.drain[d], 1);
+    }
     sm.abort = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -478,7 +618,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
     if (lane == 0) {
       uint32_t kv_it = 0, it_cnt = 0;
       bool ok = true;
-      for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+      for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+        const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+        if (k >= n_items) continue;
         int b, h, i;
         decode(k, sh, n_qt, b, h, i);
         const int slot = it_cnt & 1;
@@ -507,13 +649,15 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
+    // S = Q_i K_j^T and dP = dO_i V_j^T for every key tile j <= i.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, 64, 0, 1);
-      const uint32_t t_s = tmem + 0, t_dp = tmem + 128, t_ds0 = tmem + 256, t_dq = tmem + 384;
-      uint32_t kv_it = 0, it_cnt = 0, sdp_cnt = 0, ds_cnt = 0;
+      const uint32_t t_s = tmem + 0, t_dp = tmem + 128;
+      uint32_t kv_it = 0, it_cnt = 0, sdp_cnt = 0;
       bool ok = true;
-      for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x, ++it_cnt) {
+      for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+        const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+        if (k >= n_items) continue;
         int b, h, i;
         decode(k, sh, n_qt, b, h, i);
         const int slot = it_cnt & 1;
@@ -522,123 +666,183 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
         const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.q[slot]), 16, 1024);
         const uint64_t odesc = smem_desc_sw128(smem_u32(sm.dout[slot]), 16, 1024);
         const int n_j = i + 1;
-        auto issue_sdp = [&](uint32_t it_idx) -> bool {
-          const int s = it_idx % kStages;
-          if (!mbar_wait(&sm.kv_full[s], (it_idx / kStages) & 1, kSiteDqMma, abort)) return false;
-          if (sdp_cnt > 0 && !mbar_wait(&sm.sdp_free, (sdp_cnt - 1) & 1, kSiteDqMma, abort))
-            return false;
+        for (int n = 0; n < n_j; ++n) {
+          const uint32_t idx = kv_it + n;
+          const int s = idx % kStages;
+          if (!mbar_wait(&sm.kv_full[s], (idx / kStages) & 1, kSiteDqMma, abort)) { ok = false; break; }
+          if (sdp_cnt > 0 && !mbar_wait(&sm.sdp_free, (sdp_cnt - 1) & 1, kSiteDqMma, abort)) { ok = false; break; }
           tc_fence_after();
           const uint64_t kdesc = smem_desc_sw128(smem_u32(sm.k[s]), 16, 1024);
           const uint64_t vdesc = smem_desc_sw128(smem_u32(sm.v[s]), 16, 1024);
+          mma_ss(t_s, qdesc, kdesc, idesc_s, 0u);
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) mma_ss(t_s, qdesc + 2 * kk, kdesc + 2 * kk, idesc_s, kk > 0);
+          for (int kk = 1; kk < kD / 16; ++kk) mma_ss(t_s, qdesc + 2 * kk, kdesc + 2 * kk, idesc_s, 1u);
+          mma_ss(t_dp, odesc, vdesc, idesc_s, 0u);
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) mma_ss(t_dp, odesc + 2 * kk, vdesc + 2 * kk, idesc_s, kk > 0);
+          for (int kk = 1; kk < kD / 16; ++kk) mma_ss(t_dp, odesc + 2 * kk, vdesc + 2 * kk, idesc_s, 1u);
           mma_commit(&sm.sdp_full);
           ++sdp_cnt;
-          return true;
-        };
-        if (!issue_sdp(kv_it)) { ok = false; break; }
+        }
+        if (!ok) break;
+        kv_it += n_j;
+        ++it_cnt;
+      }
+      mma_commit(&sm.drain[0]);
+      drain_wait(&sm.drain[0], 0, kSiteDqMma);
+    }
+    __syncwarp();
+  } else if (warp == kAccWarp) {
+    // dQ += dS K_j once the elementwise step wrote dS.
+    if (lane == 0) {
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, 64, 0, 1);
+      const uint32_t t_ds0 = tmem + 256, t_dq = tmem + 384;
+      uint32_t kv_it = 0, it_cnt = 0, ds_cnt = 0;
+      bool ok = true;
+      for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+        const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+        if (k >= n_items) continue;
+        int b, h, i;
+        decode(k, sh, n_qt, b, h, i);
+        const int slot = it_cnt & 1;
+        const int n_j = i + 1;
         for (int n = 0; n < n_j; ++n) {
-          const uint32_t cur = kv_it + n;
-          if (n + 1 < n_j && !issue_sdp(cur + 1)) { ok = false; break; }
+          const uint32_t idx = kv_it + n;
+          const int s = idx % kStages;
+          // ds_full implies this stage's K landed and S/dP are done.
           if (!mbar_wait(&sm.ds_full, ds_cnt & 1, kSiteDqMma, abort)) { ok = false; break; }
-          const uint32_t t_ds = t_ds0 + 64 * (ds_cnt & 1);
+          const int buf = ds_cnt & 1;
+          const uint32_t t_ds = t_ds0 + 64 * buf;
           ++ds_cnt;
           tc_fence_after();
-          const int s = cur % kStages;
           const uint64_t kdesc_mn = smem_desc_sw128(smem_u32(sm.k[s]), 128 * 128, 1024);
+          mma_ts(t_dq, t_ds, kdesc_mn, idesc_acc, n > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < kBlockN / 16; ++kk)
-            mma_ts(t_dq, t_ds + 8 * kk, kdesc_mn + 128 * kk, idesc_acc, (n > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 1; kk < kBlockN / 16; ++kk)
+            mma_ts(t_dq, t_ds + 8 * kk, kdesc_mn + 128 * kk, idesc_acc, 1u);
+          mma_commit(&sm.ds_free[buf]);
+          // S/dP of this key tile finished before its dS was written, so the
+          // stage can be refilled once this product is done.
           mma_commit(&sm.kv_empty[s]);
         }
         if (!ok) break;
         kv_it += n_j;
         mma_commit(&sm.acc_done);
         mma_commit(&sm.in_empty[slot]);
+        ++it_cnt;
       }
-      mma_commit(&sm.drain);
-      drain_wait(&sm.drain, 0, kSiteDqMma);
+      mma_commit(&sm.drain[1]);
+      drain_wait(&sm.drain[1], 0, kSiteDqMma);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------- elementwise WGs
     const int r = ((warp & 3) << 5) + lane;  // query row within the tile = TMEM lane
-    const int g = warp >> 2;                 // key columns [64g, 64g + 64)
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
-    const uint32_t t_s = tmem + lane_base + 64 * g, t_dp = tmem + lane_base + 128 + 64 * g;
-    const uint32_t t_ds0 = tmem + lane_base + 256 + 32 * g, t_dq = tmem + lane_base + 384 + 32 * g;
+    const int g = warp >> 2;                 // key columns [32g, 32g + 32)
+    const int r_lo = (warp & 3) << 5;
+    const uint32_t lb = static_cast<uint32_t>(r_lo) << 16;
+    const uint32_t t_s = tmem + lb + 32 * g, t_dp = tmem + lb + 128 + 32 * g;
+    const uint32_t t_ds0 = tmem + lb + 256 + 16 * g, t_dq = tmem + lb + 384 + 16 * g;
+    const float sc = sh.scale_log2;
     uint32_t sdp_cnt = 0, acc_cnt = 0, ds_cnt = 0;
+    // The finished item whose dQ still sits in tensor memory: it is read out
+    // while the next item's first tile is processed, just before that tile's
+    // dS goes to tensor memory (after which the next dQ product overwrites
+    // the accumulator).
+    bool pending = false;
+    int pb = 0, ph = 0, prow = 0;
     bool ok = true;
-    for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+    for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+      const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+      if (k >= n_items) continue;
       int b, h, i;
       decode(k, sh, n_qt, b, h, i);
       const int row = i * kBlockM + r;
       const bool valid = row < sh.T;
       const size_t lrow = (static_cast<size_t>(b) * sh.H + h) * sh.T + row;
-      const float lse2 = valid ? lse[lrow] * kLog2e : INFINITY;
-      const float dlt = valid ? delta[lrow] : 0.f;
+      // Rows past T get -lse = -inf (P = 0).
+      const float nl = valid ? -lse[lrow] * kLog2e : -INFINITY;
+      const float nd = valid ? -delta[lrow] : 0.f;
       for (int j = 0; j <= i; ++j) {
         ok = mbar_wait(&sm.sdp_full, sdp_cnt & 1, kSiteDqSoftmax, abort);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++sdp_cnt;
         tc_fence_after();
-        const bool diag = (j == i);
-        const uint32_t t_ds = t_ds0 + 64 * (ds_cnt & 1);
+        const int buf = ds_cnt & 1;
+        const uint32_t t_ds = t_ds0 + 64 * buf;
+        const uint32_t uses = ds_cnt >> 1;  // earlier dS tiles written to this buffer
         ++ds_cnt;
-        uint32_t sv[64], dv[64];
-        tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sv));
-        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-        tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dv));
-        tmem_ld32(t_dp + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.sdp_free);
-        uint32_t dd[32];
+        uint32_t dd[16];
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          float ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 2 * c2 + e;
-            float x = fmaf(__uint_as_float(sv[c]), sh.scale_log2, -lse2);
-            if (diag && (64 * g + c) > r) x = -INFINITY;  // key after query
-            const float p = ex2(x);
-            ds[e] = p * (__uint_as_float(dv[c]) - dlt);
+        for (int half = 0; half < 2; ++half) {  // 16 key columns at a time
+          uint32_t sv[16], dv[16];
+          tmem_ld16(t_s + 16 * half, sv);
+          tmem_ld16(t_dp + 16 * half, dv);
+          tmem_wait_ld();
+          if (half == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.sdp_free);
           }
-          dd[c2] = pack_bf16_fast(ds[0], ds[1]);
+          const int c0 = 32 * g + 16 * half;  // first key column of the chunk
+          uint32_t (&ddh)[8] = *reinterpret_cast<uint32_t(*)[8]>(dd + 8 * half);
+          // On the diagonal tile, a chunk needs the mask if one of its keys lies
+          // after one of this warp's queries.
+          if (j == i && c0 + 15 > r_lo)
+            dq_chunk<true>(sv, dv, nl, nd, sc, c0, r, ddh);
+          else
+            dq_chunk<false>(sv, dv, nl, nd, sc, c0, r, ddh);
         }
-        tmem_st32(t_ds, dd);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.ds_full);
+        if (uses > 0) {
+          // The dQ product that read this buffer two tiles ago must be done.
+          ok = mbar_wait(&sm.ds_free[buf], (uses - 1) & 1, kSiteDqSoftmax, abort);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        if (j == 0 && pending) {
+          // Read the finished item's dQ out before this tile's dQ product
+          // overwrites it; store it once this tile is handed over.
+          ok = mbar_wait(&sm.acc_done, acc_cnt & 1, kSiteDqSoftmax, abort);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ++acc_cnt;
+          tc_fence_after();
+          uint32_t aq[16];
+          tmem_ld16(t_dq, aq);
+          tmem_wait_ld();
+          tmem_st16(t_ds, dd);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.ds_full);
+          store_dq_row(dqkv, aq, pb, ph, prow, g, C, sh);
+          pending = false;
+        } else {
+          tmem_st16(t_ds, dd);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.ds_full);
+        }
       }
       if (!ok) break;
+      pending = true;
+      pb = b;
+      ph = h;
+      prow = row;
+    }
+    if (ok && pending) {
       ok = mbar_wait(&sm.acc_done, acc_cnt & 1, kSiteDqSoftmax, abort);
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      ++acc_cnt;
-      tc_fence_after();
-      // Warpgroup g stores d columns [32g, 32g + 32) of dQ.
-      uint32_t a[32];
-      tmem_ld32(t_dq, a);
-      tmem_wait_ld();
-      tc_fence_before();
-      if (valid) {
-        const float sc = sh.scale;
-        uint4* dst = reinterpret_cast<uint4*>(dqkv + ((static_cast<size_t>(b) * sh.T + row) * 3) * C +
-                                              h * kD + 32 * g);
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          dst[v] = make_uint4(
-              pack_bf16(__uint_as_float(a[8 * v]) * sc, __uint_as_float(a[8 * v + 1]) * sc),
-              pack_bf16(__uint_as_float(a[8 * v + 2]) * sc, __uint_as_float(a[8 * v + 3]) * sc),
-              pack_bf16(__uint_as_float(a[8 * v + 4]) * sc, __uint_as_float(a[8 * v + 5]) * sc),
-              pack_bf16(__uint_as_float(a[8 * v + 6]) * sc, __uint_as_float(a[8 * v + 7]) * sc));
+      if (ok) {
+        ++acc_cnt;
+        tc_fence_after();
+        uint32_t aq[16];
+        tmem_ld16(t_dq, aq);
+        tmem_wait_ld();
+        tc_fence_before();
+        store_dq_row(dqkv, aq, pb, ph, prow, g, C, sh);
       }
     }
   }

@@ -7,19 +7,26 @@
 //
 //   * Work item = one (batch, head) and a pair of adjacent 128-row query tiles
 //     (rows [256p, 256p+256)). Items run heaviest first over a persistent grid.
-//   * Warp 8 (TMA): loads the two Q tiles once per item (double-buffered
+//   * Warp 16 (TMA): loads the two Q tiles once per item (double-buffered
 //     across items) and streams the 128-row K and V tiles j = 0..2p+1 through a
 //     4-stage shared-memory ring.
-//   * Warp 9 (MMA, one thread): S_q = Q_q K_j^T (M128 N128 K64) into tensor
-//     memory, then O_q += P_q V_j (M128 N64 K128) with P_q read from tensor
-//     memory. Key tiles above the diagonal are never issued.
-//   * Warps 0-3 and 4-7 (softmax, one warpgroup per query tile, one row per
-//     thread): load the S row from tensor memory, apply the causal mask on the
-//     diagonal tile, run the online softmax in base 2 (running max m, running
-//     sum l), rescale O in tensor memory when m grows, and write P as fp16 back
-//     to tensor memory. At the end they normalise O, store out (bf16) and
-//     lse = ln2 * (m + log2 l).
-//   * Warps 10-11 (convert): rewrite each V tile in shared memory from bf16 to
+//   * Warps 17 and 18 (MMA, one thread each, one per query tile q): S_q = Q_q
+//     K_j^T (M128 N128 K64) into tensor memory, issued for key tile j+1 as soon
+//     as the softmax has read S_q(j), then O_q += P_q V_j (M128 N64 K128) with
+//     P_q read from tensor memory. Key tiles above the diagonal are never
+//     issued. Each query tile has its own issuing thread, so neither waits on
+//     the other tile's softmax.
+//   * Warps 0-15 (softmax): four warpgroups; warpgroup w serves query tile
+//     q = w / 2 and key columns [64h, 64h + 64) of every key tile, h = w % 2.
+//     Each thread owns one query row (its TMEM lane) and half of its columns:
+//     it loads them from tensor memory, applies the causal mask on the
+//     diagonal tile, exchanges its partial row max with the thread holding the
+//     other half (shared memory, double-buffered, mbarrier-synchronised), runs
+//     the online softmax in base 2 (running max m, partial running sum l),
+//     rescales its half of O in tensor memory when m grows, and writes its half
+//     of P as fp16. At the end the two partial sums are combined, O is
+//     normalised and stored (bf16), and lse = ln2 * (m + log2 l) is written.
+//   * Warp 19 (convert): rewrites each V tile in shared memory from bf16 to
 //     fp16 in place, so that O += P V runs as an fp16 x fp16 product. P in
 //     [0, 1] keeps 11 significant bits instead of 8, which matters on peaked
 //     rows where one probability near 1 multiplies a large v. Every bf16 value
@@ -28,10 +35,7 @@
 //
 // Tensor memory (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256),
 // P_0 [256,320), P_1 [320,384) (fp16 pairs), O_0 [384,448), O_1 [448,512).
-//
-// Registers: 384 threads launch with 168 each; the producer/MMA/convert
-// warpgroup drops to 88 and the two softmax warpgroups rise to 208
-// (128*88 + 256*208 = 384*168).
+
 #pragma once
 
 #include "common.cuh"
@@ -41,22 +45,15 @@ namespace ga {
 namespace fwd {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 384;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kConvertWarp0 = 10;  // warps 10 and 11
-// Register split (setmaxnreg): the producer/MMA/convert warpgroup gives up
-// registers to the two softmax warpgroups. The total must fit the block's
-// launch allocation (kThreads x kLaunchRegs), or setmaxnreg.inc would wait
-// forever; the host checks the compiled register count before any launch.
-constexpr uint32_t kLaunchRegs = 168;
+constexpr int kThreads = 640;
+constexpr int kSoftmaxWarps = 16;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;      // issues for query tile 0, owns the TMEM allocation
+constexpr int kMmaWarp1 = 18;     // issues for query tile 1
+constexpr int kConvertWarp = 19;
 // The running max is raised only when a row's max grows by more than this many
 // powers of two; until then P may reach 2^8 (well inside fp16).
 constexpr float kRescaleLog2 = 8.f;
-constexpr uint32_t kRegsAux = 88;
-constexpr uint32_t kRegsSoftmax = 208;
-static_assert(128 * kRegsAux + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 
 __device__ __forceinline__ uint32_t col_s(int q) { return q * 128; }
@@ -70,7 +67,12 @@ struct alignas(1024) Smem {
   uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[kStages], kv_empty[kStages], v_ready[kStages];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
-  uint64_t drain;
+  uint64_t drain[2];
+  // Exchange of partial row maxima (per query tile, double-buffered) and of
+  // partial row sums between the two column halves of each row.
+  float xmax[2][2][2][kBlockM];  // [q][buffer][half][row]
+  float xsum[2][2][kBlockM];     // [q][half][row]
+  uint64_t xbar[2][2], lbar[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -100,6 +102,43 @@ __host__ __device__ __forceinline__ int num_items(const AttnShape& sh) {
   return sh.B * sh.H * ceil_div(ceil_div(sh.T, kBlockM), 2);
 }
 
+// Epilogue of one query row for one column half: combines the two halves'
+// partial sums through shared memory, normalises this half of O (already
+// loaded from tensor memory) and stores it as bf16; half 0 writes
+// lse = ln2 * (m*c + log2 l). Returns false if the exchange wait gave up.
+__device__ __forceinline__ bool finish_row(Smem& sm, int q, int hf, int r, int lane,
+                                           uint32_t& l_cnt, volatile int* abort,
+                                           const uint32_t (&o)[32], int b, int h, int row,
+                                           float m, float l, __nv_bfloat16* __restrict__ out,
+                                           float* __restrict__ lse, const AttnShape& sh) {
+  sm.xsum[q][hf][r] = l;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&sm.lbar[q]);
+  bool ok = mbar_wait(&sm.lbar[q], l_cnt & 1, kSiteFwdSoftmax, abort);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) return false;
+  ++l_cnt;
+  l += sm.xsum[q][hf ^ 1][r];
+  if (row < sh.T) {
+    const float inv_l = 1.f / l;
+    uint4* dst = reinterpret_cast<uint4*>(
+        out + ((static_cast<size_t>(b) * sh.T + row) * sh.H + h) * kD + 32 * hf);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint4 w;
+      w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+      w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+      w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+      w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+      dst[v] = w;
+    }
+    if (hf == 0)
+      lse[(static_cast<size_t>(b) * sh.H + h) * sh.T + row] =
+          (m * sh.scale_log2 + lg2(l)) * 0.69314718055994531f;
+  }
+  return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __restrict__ out,
                 float* __restrict__ lse, const AttnShape sh) {
@@ -115,20 +154,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.q_full[s], 1);
-      mbar_init(&sm.q_empty[s], 1);
+      mbar_init(&sm.q_empty[s], 2);   // one arrival per issuing thread
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 2);  // one arrival per query tile of the item
-      mbar_init(&sm.v_ready[s], 2);   // one arrival per convert warp
+      mbar_init(&sm.v_ready[s], 1);
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(&sm.s_full[q], 1);
-      mbar_init(&sm.s_free[q], 4);
-      mbar_init(&sm.p_full[q], 4);
+      mbar_init(&sm.s_free[q], 8);   // the 8 softmax warps of the query tile
+      mbar_init(&sm.p_full[q], 8);
       mbar_init(&sm.o_done[q], 1);
+      mbar_init(&sm.drain[q], 1);
+      mbar_init(&sm.xbar[q][0], 8);
+      mbar_init(&sm.xbar[q][1], 8);
+      mbar_init(&sm.lbar[q], 8);
     }
-    mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -142,13 +184,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp >= kProducerWarp) {
-  regs_dealloc<kRegsAux>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA warp
     if (lane == 0) {
       uint32_t kv_it = 0, it_cnt = 0;
-      for (int k = blockIdx.x; k < n_items; k += gridDim.x) {
+      for (int rnd = 0; rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+        const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+        if (k >= n_items) continue;
         const Item it = decode_item(k, sh);
         const int slot = it_cnt & 1;
         if (!mbar_wait(&sm.q_empty[slot], ((it_cnt >> 1) & 1) ^ 1, kSiteFwdProducer, abort)) break;
@@ -181,106 +223,91 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
           drain_wait(&sm.q_full[s], ((it_cnt - s + 1) / 2 - 1) & 1, kSiteFwdProducer);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA warp
-    // Event-driven issue: the two query tiles of an item advance
-    // independently. Whenever a tile's next S product is possible (its key
-    // tile has landed and its softmax has read the previous S) or its next
-    // P V product is possible (P written, V converted), it is issued. One
-    // query tile therefore never waits on the other tile's softmax.
+  } else if (warp == kMmaWarp || warp == kMmaWarp1) {
+    // ------------------------------------------------------------ MMA warps
+    // One issuing thread per query tile q. Per item: S_q(0); then for each
+    // key tile j the thread issues S_q(j+1) once the softmax has read S_q(j),
+    // then O_q += P_q(j) V_j once P_q(j) is written and V_j converted.
+    const int q = warp - kMmaWarp;
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_o = idesc_f16_f32(128, 64, 0, 1);
-      uint32_t kv_it = 0, it_cnt = 0;
-      uint32_t s_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+      const uint32_t t_s = tmem + col_s(q), t_p = tmem + col_p(q), t_o = tmem + col_o(q);
+      uint32_t kv_it = 0, it_cnt = 0, s_cnt = 0, p_cnt = 0;
       bool ok = true;
-      for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x, ++it_cnt) {
+      for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+        const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+        if (k >= n_items) continue;
         const Item it = decode_item(k, sh);
         const int slot = it_cnt & 1;
-        if (!mbar_wait(&sm.q_full[slot], (it_cnt >> 1) & 1, kSiteFwdMma, abort)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t qdesc[2] = {smem_desc_sw128(smem_u32(sm.q[slot][0]), 16, 1024),
-                                   smem_desc_sw128(smem_u32(sm.q[slot][1]), 16, 1024)};
-        // Key tiles seen by each query tile: 0..i0 and 0..i0+1 (if it exists).
-        const int n_tiles[2] = {it.i0 + 1, it.has1 ? it.i0 + 2 : 0};
-        int ns[2] = {0, 0}, np[2] = {0, 0};
-        // A stage is released by two arrivals, one per query tile. When only
-        // one query tile uses a key tile, issuing its P V product also makes
-        // the other tile's arrival (never earlier: an early arrival could
-        // complete the stage's previous phase).
-        uint64_t t_idle = 0;
-        while (np[0] < n_tiles[0] || np[1] < n_tiles[1]) {
-          bool progressed = false;
+        // Key tiles this query tile sees, and those the other one sees.
+        const int n = q == 0 ? it.i0 + 1 : (it.has1 ? it.i0 + 2 : 0);
+        const int n_other = q == 0 ? (it.has1 ? it.i0 + 2 : 0) : it.i0 + 1;
+        if (n == 0) {
+          // No second query tile in this item: this thread still releases its
+          // share of the Q slot, after the slot's previous phase is complete
+          // (an earlier arrival could complete that phase instead).
+          if (!mbar_wait(&sm.q_empty[slot], ((it_cnt >> 1) & 1) ^ 1, kSiteFwdMma, abort)) { ok = false; break; }
+          mbar_arrive(&sm.q_empty[slot]);
+        } else {
+          if (!mbar_wait(&sm.q_full[slot], (it_cnt >> 1) & 1, kSiteFwdMma, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.q[slot][q]), 16, 1024);
+          // S_q(jj) = Q_q K(jj)^T, K = 64 in steps of 16 (32 bytes).
+          auto issue_s = [&](int jj) -> bool {
+            const uint32_t idx = kv_it + jj;
+            const int st = idx % kStages;
+            if (!mbar_wait(&sm.kv_full[st], (idx / kStages) & 1, kSiteFwdMma, abort)) return false;
+            if (s_cnt > 0 && !mbar_wait(&sm.s_free[q], (s_cnt - 1) & 1, kSiteFwdMma, abort)) return false;
+            tc_fence_after();
+            const uint64_t kdesc = smem_desc_sw128(smem_u32(sm.k[st]), 16, 1024);
+            mma_ss(t_s, qdesc, kdesc, idesc_s, 0u);
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            // S_q(j) = Q_q K_j^T: needs K_j and the S_q buffer free.
-            if (ns[q] < n_tiles[q] && ns[q] <= np[q] + 1) {
-              const uint32_t idx = kv_it + ns[q];
-              const int st = idx % kStages;
-              if (mbar_test(&sm.kv_full[st], (idx / kStages) & 1) &&
-                  (s_cnt[q] == 0 || mbar_test(&sm.s_free[q], (s_cnt[q] - 1) & 1))) {
-                tc_fence_after();
-                const uint64_t kdesc = smem_desc_sw128(smem_u32(sm.k[st]), 16, 1024);
+            for (int kk = 1; kk < kD / 16; ++kk) mma_ss(t_s, qdesc + 2 * kk, kdesc + 2 * kk, idesc_s, 1u);
+            mma_commit(&sm.s_full[q]);
+            ++s_cnt;
+            return true;
+          };
+          if (!issue_s(0)) { ok = false; break; }
+          for (int j = 0; j < n; ++j) {
+            if (j + 1 < n && !issue_s(j + 1)) { ok = false; break; }
+            const uint32_t idx = kv_it + j;
+            const int st = idx % kStages;
+            if (!mbar_wait(&sm.p_full[q], p_cnt & 1, kSiteFwdMma, abort)) { ok = false; break; }
+            ++p_cnt;
+            if (!mbar_wait(&sm.v_ready[st], (idx / kStages) & 1, kSiteFwdMma, abort)) { ok = false; break; }
+            tc_fence_after();
+            // 16 keys = 8 TMEM columns of P and 2048 bytes of V per step.
+            const uint64_t vdesc = smem_desc_sw128(smem_u32(sm.v[st]), 128 * 128, 1024);
+            mma_ts(t_o, t_p, vdesc, idesc_o, j > 0 ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)  // K = 64 in steps of 16 (32 bytes)
-                  mma_ss(tmem + col_s(q), qdesc[q] + 2 * kk, kdesc + 2 * kk, idesc_s, kk > 0);
-                mma_commit(&sm.s_full[q]);
-                ++s_cnt[q];
-                ++ns[q];
-                progressed = true;
-              }
-            }
-            // O_q += P_q(j) V_j: needs P_q(j) written and V_j converted.
-            if (np[q] < ns[q]) {
-              const uint32_t idx = kv_it + np[q];
-              const int st = idx % kStages;
-              if (mbar_test(&sm.p_full[q], p_cnt[q] & 1) &&
-                  mbar_test(&sm.v_ready[st], (idx / kStages) & 1)) {
-                tc_fence_after();
-                const uint64_t vdesc = smem_desc_sw128(smem_u32(sm.v[st]), 128 * 128, 1024);
-                // 16 keys = 8 TMEM columns of P and 2048 bytes of V per step.
-#pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk)
-                  mma_ts(tmem + col_o(q), tmem + col_p(q) + 8 * kk, vdesc + 128 * kk, idesc_o,
-                         (np[q] > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&sm.o_done[q]);
-                mma_commit(&sm.kv_empty[st]);
-                if (np[q] >= n_tiles[1 - q]) mbar_arrive(&sm.kv_empty[st]);
-                ++p_cnt[q];
-                ++np[q];
-                progressed = true;
-              }
-            }
+            for (int kk = 1; kk < kBlockN / 16; ++kk)
+              mma_ts(t_o, t_p + 8 * kk, vdesc + 128 * kk, idesc_o, 1u);
+            mma_commit(&sm.o_done[q]);
+            // The stage is released by two arrivals. A key tile the other query
+            // tile does not see gets its second arrival here (its previous
+            // phase is complete: this thread saw the tile land).
+            mma_commit(&sm.kv_empty[st]);
+            if (j >= n_other) mbar_arrive(&sm.kv_empty[st]);
           }
-          if (progressed) {
-            t_idle = 0;
-          } else if (t_idle == 0) {
-            t_idle = globaltimer();
-          } else if (*abort) {
-            ok = false;
-            break;
-          } else if (globaltimer() - t_idle > kWaitTimeoutNs) {
-            record_failure(kSiteFwdMma);
-            *abort = 1;
-            ok = false;
-            break;
-          }
+          if (!ok) break;
+          mma_commit(&sm.q_empty[slot]);
         }
-        if (!ok) break;
         kv_it += it.n_kv;
-        mma_commit(&sm.q_empty[slot]);
+        ++it_cnt;
       }
       // Drain: every MMA this thread issued has finished before TMEM is freed.
-      mma_commit(&sm.drain);
-      drain_wait(&sm.drain, 0, kSiteFwdMma);
+      mma_commit(&sm.drain[q]);
+      drain_wait(&sm.drain[q], 0, kSiteFwdMma);
     }
     __syncwarp();
-  } else if (warp >= kConvertWarp0) {
+  } else if (warp == kConvertWarp) {
     // ------------------------------------------------------------ convert V
-    const int ct = threadIdx.x - kConvertWarp0 * 32;  // 0..63
     uint32_t kv_it = 0;
     bool ok = true;
-    for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+    for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+      const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+      if (k >= n_items) continue;
       const Item it = decode_item(k, sh);
       for (int j = 0; j < it.n_kv; ++j, ++kv_it) {
         const int s = kv_it % kStages;
@@ -290,13 +317,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         uint4* tile = reinterpret_cast<uint4*>(sm.v[s]);
         bool bad = false;
 #pragma unroll 4
-        for (int c = ct; c < kTileBytes / 16; c += 64) {
+        for (int c = lane; c < kTileBytes / 16; c += 32) {
           uint4 w = tile[c];
           uint32_t* u = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             bad |= bf16x2_out_of_f16_range(u[e]) != 0;
-            u[e] = bf16x2_to_f16x2(u[e]);
+            // bf16 -> fp32 is exact (a shift); fp32 -> fp16 rounds to nearest,
+            // exact for every bf16 value with |v| <= 65504 except fp16
+            // subnormals (|v| < 6.1e-5, within 3e-8).
+            u[e] = pack_f16(__uint_as_float(u[e] << 16), __uint_as_float(u[e] & 0xFFFF0000u));
           }
           tile[c] = w;
         }
@@ -304,30 +334,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         // Generic-proxy stores must be visible to the tensor core (async proxy).
         fence_proxy_async_smem();
         __syncwarp();
-        if ((ct & 31) == 0) mbar_arrive(&sm.v_ready[s]);
+        if (lane == 0) mbar_arrive(&sm.v_ready[s]);
       }
     }
-  }
   } else {
-    regs_alloc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
-    const int q = warp >> 2;                       // query tile of the pair
+    const int q = warp >> 3;                       // query tile of the pair
+    const int hf = (warp >> 2) & 1;                // column half [64hf, 64hf + 64)
     const int r = ((warp & 3) << 5) + lane;        // row within the tile = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
-    const uint32_t t_s = tmem + lane_base + col_s(q);
-    const uint32_t t_p = tmem + lane_base + col_p(q);
-    const uint32_t t_o = tmem + lane_base + col_o(q);
-    uint32_t s_cnt = 0, o_cnt = 0;
+    const uint32_t t_s = tmem + lane_base + col_s(q) + 64 * hf;
+    const uint32_t t_p = tmem + lane_base + col_p(q) + 32 * hf;
+    const uint32_t t_o = tmem + lane_base + col_o(q) + 32 * hf;
+    uint32_t s_cnt = 0, o_cnt = 0, x_cnt = 0, l_cnt = 0;
+    // The finished item whose O still sits in tensor memory. It is read out
+    // while the next item's first tile is processed, just before that tile's
+    // P goes to tensor memory (the next P V product then overwrites O); the
+    // normalisation and stores follow once that tile is handed over.
+    bool pending = false;
+    int p_b = 0, p_h = 0, p_row = 0;
+    float p_m = 0.f, p_l = 0.f;
     bool ok = true;
-    for (int k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+    for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
+      const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+      if (k >= n_items) continue;
       const Item it = decode_item(k, sh);
       if (q == 1 && !it.has1) continue;
       const int i = it.i0 + q;
       const int row = i * kBlockM + r;
-      // Running max m (raw logit units, as read from S) and running sum l of
-      // 2^(s*c - m*c), c = scale*log2(e). m is only raised when the row max
-      // grows by more than kRescaleLog2 in log2 units; until then P and l keep
-      // using the stale m, which stays exact because O / l uses the same m.
+      // Running max m (raw logit units, as read from S) and this half's running
+      // sum l of 2^(s*c - m*c), c = scale*log2(e). m is only raised when the
+      // row max grows by more than kRescaleLog2 in log2 units; until then P and
+      // l keep using the stale m, which stays exact because O / l uses the
+      // same m. Both halves of a row always hold the same m.
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j <= i; ++j) {
         ok = mbar_wait(&sm.s_full[q], s_cnt & 1, kSiteFwdSoftmax, abort);
@@ -335,46 +374,58 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
-        float x[128];
+        float x[64];
         {
-          uint32_t u[128];
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tmem_ld32(t_s + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(u + 32 * c));
+          uint32_t u[64];
+          tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(u));
+          tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
+          for (int e = 0; e < 64; ++e) x[e] = __uint_as_float(u[e]);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_free[q]);
 
         if (j == i) {
-          const int lim = row - j * kBlockN;  // columns c > lim are future keys
+          const int lim = row - j * kBlockN - 64 * hf;  // columns c > lim are future keys
 #pragma unroll
-          for (int c = 0; c < 128; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
+          for (int c = 0; c < 64; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
         }
-        // Row max: 8 independent chains of 3-input max.
+        // Partial row max: 8 independent chains of 3-input max.
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = fmax3(x[e], x[8 + e], x[16 + e]);
 #pragma unroll
-        for (int c = 24; c < 128; c += 16) {
+        for (int c = 24; c < 56; c += 16) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], x[c + e], x[c + 8 + e]);
         }
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                               fmaxf(mx8[6], mx8[7]));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[56 + e]);
+        float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                         fmaxf(mx8[6], mx8[7]));
+        // Exchange with the other half of the row.
+        {
+          const int buf = x_cnt & 1;
+          sm.xmax[q][buf][hf][r] = mx;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.xbar[q][buf]);
+          ok = mbar_wait(&sm.xbar[q][buf], (x_cnt >> 1) & 1, kSiteFwdSoftmax, abort);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ++x_cnt;
+          mx = fmaxf(mx, sm.xmax[q][buf][hf ^ 1][r]);
+        }
         const bool grow = (mx - m) * sh.scale_log2 > kRescaleLog2;  // always true on j == 0
         const float m_new = grow ? mx : m;
         const float alpha = grow ? ex2((m - m_new) * sh.scale_log2) : 1.f;
         const float neg_mc = -m_new * sh.scale_log2;
-        // p = 2^(s*c - m*c), row sum, and fp16 packing of P in one pass, so the
-        // packing runs in the shadow of the exp2 calls.
-        uint32_t pk[64];
+        // p = 2^(s*c - m*c), partial row sum, and fp16 packing of P in one pass.
+        uint32_t pk[32];
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c2 = 0; c2 < 64; ++c2) {
+        for (int c2 = 0; c2 < 32; ++c2) {
           float y0, y1;
           fma2(x[2 * c2], x[2 * c2 + 1], sh.scale_log2, neg_mc, y0, y1);
           const float p0 = ex2(y0), p1 = ex2(y1);
@@ -385,60 +436,64 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         l = l * alpha + sum;
         m = m_new;
 
-        if (j > 0) {
-          // O must hold P_{j-1} V_{j-1} before it is rescaled and P is reused.
+        const bool flush = (j == 0) && pending;
+        if (j > 0 || flush) {
+          // O must hold P_{j-1} V_{j-1} (or the finished item's last product)
+          // before it is rescaled or read, and before P is reused.
           ok = mbar_wait(&sm.o_done[q], o_cnt & 1, kSiteFwdSoftmax, abort);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ++o_cnt;
           tc_fence_after();
-          if (__any_sync(0xffffffffu, grow)) {
-            uint32_t o[64];
-            tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(o));
-            tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+          if (!flush && __any_sync(0xffffffffu, grow)) {
+            uint32_t oo[32];
+            tmem_ld32(t_o, oo);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(t_o, *reinterpret_cast<uint32_t(*)[32]>(o));
-            tmem_st32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+            for (int e = 0; e < 32; ++e) oo[e] = __float_as_uint(__uint_as_float(oo[e]) * alpha);
+            tmem_st32(t_o, oo);
             tmem_wait_st();
           }
         }
-        tmem_st32(t_p, *reinterpret_cast<uint32_t(*)[32]>(pk));
-        tmem_st32(t_p + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+        tmem_st32(t_p, pk);
         tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.p_full[q]);
+        if (flush) {
+          // The finished item's O is read before this tile's P V product (which
+          // starts only after the arrival below) overwrites it.
+          uint32_t o[32];
+          tmem_ld32(t_o, o);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.p_full[q]);
+          ok = finish_row(sm, q, hf, r, lane, l_cnt, abort, o, p_b, p_h, p_row, p_m, p_l, out, lse, sh);
+          if (!ok) break;
+          pending = false;
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.p_full[q]);
+        }
       }
       if (!ok) break;
-
-      // Epilogue: O / l -> out (bf16), lse in natural log.
+      pending = true;
+      p_b = it.b;
+      p_h = it.h;
+      p_row = row;
+      p_m = m;
+      p_l = l;
+    }
+    if (ok && pending) {
       ok = mbar_wait(&sm.o_done[q], o_cnt & 1, kSiteFwdSoftmax, abort);
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      ++o_cnt;
-      tc_fence_after();
-      uint32_t o[64];
-      tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(o));
-      tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
-      tmem_wait_ld();
-      tc_fence_before();
-      if (row < sh.T) {
-        const float inv_l = 1.f / l;
-        uint4* dst = reinterpret_cast<uint4*>(
-            out + ((static_cast<size_t>(it.b) * sh.T + row) * sh.H + it.h) * kD);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          uint4 w;
-          w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-          w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-          w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-          w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-          dst[v] = w;
-        }
-        lse[(static_cast<size_t>(it.b) * sh.H + it.h) * sh.T + row] =
-            (m * sh.scale_log2 + lg2(l)) * 0.69314718055994531f;
+      if (ok) {
+        ++o_cnt;
+        tc_fence_after();
+        uint32_t o[32];
+        tmem_ld32(t_o, o);
+        tmem_wait_ld();
+        tc_fence_before();
+        finish_row(sm, q, hf, r, lane, l_cnt, abort, o, p_b, p_h, p_row, p_m, p_l, out, lse, sh);
       }
     }
   }

@@ -222,6 +222,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      GA_W8(0)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -336,6 +343,30 @@ __device__ __forceinline__ void fma2(float a0, float a1, float b, float c, float
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
+// (a0 * b0 + c0, a1 * b1 + c1) in one packed fp32 fused multiply-add.
+__device__ __forceinline__ void fma2v(float a0, float a1, float b0, float b1, float c0, float c1,
+                                      float& r0, float& r1) {
+  asm("{\n\t.reg .b64 a, b, c, r;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "mov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 r, a, b, c;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// (a0 * b0, a1 * b1) in one packed fp32 multiply.
+__device__ __forceinline__ void mul2v(float a0, float a1, float b0, float b1, float& r0, float& r1) {
+  asm("{\n\t.reg .b64 a, b, r;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 r, a, b;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // (a0 + b0, a1 + b1) in one packed fp32 add.
 __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
   asm("{\n\t.reg .b64 a, b;\n\t"
@@ -390,18 +421,6 @@ __device__ __forceinline__ uint32_t bf16x2_out_of_f16_range(uint32_t w) {
 // (differs from round-to-nearest-even only on exact ties).
 __device__ __forceinline__ uint32_t pack_bf16_fast(float lo, float hi) {
   return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
-// Warpgroup-wide register budget changes (all four warps of a warpgroup
-// execute the same one). The sum over warpgroups never exceeds the block's
-// launch allocation.
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_dealloc() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_alloc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
 // Named barrier among `nthreads` threads (a multiple of 32) of the CTA.
