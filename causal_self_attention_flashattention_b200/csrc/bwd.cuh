@@ -118,8 +118,8 @@ __device__ __forceinline__ void dkdv_chunk(const uint32_t (&sv)[16], const uint3
       t1 = __uint_as_float(dv[c + 1]);
       add2(t0, t1, h ? Dl.z : Dl.x, h ? Dl.w : Dl.y);
       mul2v(p0, p1, t0, t1, d0, d1);
-      pp[c >> 1] = pack_bf16_fast(p0, p1);
-      dd[c >> 1] = pack_bf16_fast(d0, d1);
+      pp[c >> 1] = pack_bf16(p0, p1);
+      dd[c >> 1] = pack_bf16(d0, d1);
     }
   }
 }
@@ -143,7 +143,7 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[16], const uint32_
     float t0 = __uint_as_float(dv[c]), t1 = __uint_as_float(dv[c + 1]);
     add2(t0, t1, nd, nd);
     mul2v(p0, p1, t0, t1, d0, d1);
-    dd[c >> 1] = pack_bf16_fast(d0, d1);
+    dd[c >> 1] = pack_bf16(d0, d1);
   }
 }
 
