@@ -7,26 +7,23 @@
 //
 //   * Work item = one (batch, head) and a pair of adjacent 128-row query tiles
 //     (rows [256p, 256p+256)). Items run heaviest first over a persistent grid.
-//   * Warp 16 (TMA): loads the two Q tiles once per item (double-buffered
+//   * Warp 8 (TMA): loads the two Q tiles once per item (double-buffered
 //     across items) and streams the 128-row K and V tiles j = 0..2p+1 through a
 //     4-stage shared-memory ring.
-//   * Warps 17 and 18 (MMA, one thread each, one per query tile q): S_q = Q_q
+//   * Warps 9 and 10 (MMA, one thread each, one per query tile q): S_q = Q_q
 //     K_j^T (M128 N128 K64) into tensor memory, issued for key tile j+1 as soon
 //     as the softmax has read S_q(j), then O_q += P_q V_j (M128 N64 K128) with
 //     P_q read from tensor memory. Key tiles above the diagonal are never
 //     issued. Each query tile has its own issuing thread, so neither waits on
 //     the other tile's softmax.
-//   * Warps 0-15 (softmax): four warpgroups; warpgroup w serves query tile
-//     q = w / 2 and key columns [64h, 64h + 64) of every key tile, h = w % 2.
-//     Each thread owns one query row (its TMEM lane) and half of its columns:
-//     it loads them from tensor memory, applies the causal mask on the
-//     diagonal tile, exchanges its partial row max with the thread holding the
-//     other half (shared memory, double-buffered, mbarrier-synchronised), runs
-//     the online softmax in base 2 (running max m, partial running sum l),
-//     rescales its half of O in tensor memory when m grows, and writes its half
-//     of P as fp16. At the end the two partial sums are combined, O is
-//     normalised and stored (bf16), and lse = ln2 * (m + log2 l) is written.
-//   * Warp 19 (convert): rewrites each V tile in shared memory from bf16 to
+//   * Warps 0-7 (softmax): two warpgroups, warpgroup q serves query tile q.
+//     Each thread owns one query row (its TMEM lane) and all 128 columns of
+//     every key tile: it loads the row of S from tensor memory, applies the
+//     causal mask on the diagonal tile, runs the online softmax in base 2
+//     (running max m, running sum l), rescales O in tensor memory when m
+//     grows, and writes P as fp16. No row statistic crosses a thread. At the
+//     end O is normalised and stored (bf16), and lse = ln2 * (m + log2 l).
+//   * Warp 11 (convert): rewrites each V tile in shared memory from bf16 to
 //     fp16 in place, so that O += P V runs as an fp16 x fp16 product. P in
 //     [0, 1] keeps 11 significant bits instead of 8, which matters on peaked
 //     rows where one probability near 1 multiplies a large v. Every bf16 value
@@ -45,12 +42,22 @@ namespace ga {
 namespace fwd {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 640;
-constexpr int kSoftmaxWarps = 16;
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;      // issues for query tile 0, owns the TMEM allocation
-constexpr int kMmaWarp1 = 18;     // issues for query tile 1
-constexpr int kConvertWarp = 19;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;       // issues for query tile 0, owns the TMEM allocation
+constexpr int kMmaWarp1 = 10;     // issues for query tile 1
+constexpr int kConvertWarp = 11;
+// Register split (setmaxnreg): the TMA/MMA/convert warpgroup (warps 8-11) gives
+// registers to the two softmax warpgroups, which hold a whole 128-column row
+// of S. The total fits the block's launch allocation (kThreads x kLaunchRegs);
+// the host refuses to launch if the kernel was compiled for fewer registers.
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kRegsAux = 88;
+constexpr uint32_t kRegsSoftmax = 208;
+static_assert(128 * kRegsAux + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+static_assert(kProducerWarp == 8 && kConvertWarp == 11, "warps 8-11 form the aux warpgroup");
 // The running max is raised only when a row's max grows by more than this many
 // powers of two; until then P may reach 2^8 (well inside fp16).
 constexpr float kRescaleLog2 = 8.f;
@@ -68,11 +75,6 @@ struct alignas(1024) Smem {
   uint64_t kv_full[kStages], kv_empty[kStages], v_ready[kStages];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
   uint64_t drain[2];
-  // Exchange of partial row maxima (per query tile, double-buffered) and of
-  // partial row sums between the two column halves of each row.
-  float xmax[2][2][2][kBlockM];  // [q][buffer][half][row]
-  float xsum[2][2][kBlockM];     // [q][half][row]
-  uint64_t xbar[2][2], lbar[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -102,41 +104,25 @@ __host__ __device__ __forceinline__ int num_items(const AttnShape& sh) {
   return sh.B * sh.H * ceil_div(ceil_div(sh.T, kBlockM), 2);
 }
 
-// Epilogue of one query row for one column half: combines the two halves'
-// partial sums through shared memory, normalises this half of O (already
-// loaded from tensor memory) and stores it as bf16; half 0 writes
-// lse = ln2 * (m*c + log2 l). Returns false if the exchange wait gave up.
-__device__ __forceinline__ bool finish_row(Smem& sm, int q, int hf, int r, int lane,
-                                           uint32_t& l_cnt, volatile int* abort,
-                                           const uint32_t (&o)[32], int b, int h, int row,
-                                           float m, float l, __nv_bfloat16* __restrict__ out,
-                                           float* __restrict__ lse, const AttnShape& sh) {
-  sm.xsum[q][hf][r] = l;
-  __syncwarp();
-  if (lane == 0) mbar_arrive(&sm.lbar[q]);
-  bool ok = mbar_wait(&sm.lbar[q], l_cnt & 1, kSiteFwdSoftmax, abort);
-  ok = __all_sync(0xffffffffu, ok);
-  if (!ok) return false;
-  ++l_cnt;
-  l += sm.xsum[q][hf ^ 1][r];
-  if (row < sh.T) {
-    const float inv_l = 1.f / l;
-    uint4* dst = reinterpret_cast<uint4*>(
-        out + ((static_cast<size_t>(b) * sh.T + row) * sh.H + h) * kD + 32 * hf);
+// Epilogue of one query row: normalises its O (64 fp32 values read from
+// tensor memory), stores it as bf16 and writes lse = ln2 * (m*c + log2 l).
+__device__ __forceinline__ void store_row(const uint32_t (&o)[64], int b, int h, int row, float m,
+                                          float l, __nv_bfloat16* __restrict__ out,
+                                          float* __restrict__ lse, const AttnShape& sh) {
+  if (row >= sh.T) return;
+  const float inv_l = 1.f / l;
+  uint4* dst = reinterpret_cast<uint4*>(out + ((static_cast<size_t>(b) * sh.T + row) * sh.H + h) * kD);
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      uint4 w;
-      w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-      w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-      w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-      w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-      dst[v] = w;
-    }
-    if (hf == 0)
-      lse[(static_cast<size_t>(b) * sh.H + h) * sh.T + row] =
-          (m * sh.scale_log2 + lg2(l)) * 0.69314718055994531f;
+  for (int v = 0; v < 8; ++v) {
+    uint4 w;
+    w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+    w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+    w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+    w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+    dst[v] = w;
   }
-  return true;
+  lse[(static_cast<size_t>(b) * sh.H + h) * sh.T + row] =
+      (m * sh.scale_log2 + lg2(l)) * 0.69314718055994531f;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -163,13 +149,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(&sm.s_full[q], 1);
-      mbar_init(&sm.s_free[q], 8);   // the 8 softmax warps of the query tile
-      mbar_init(&sm.p_full[q], 8);
+      mbar_init(&sm.s_free[q], 4);   // the 4 softmax warps of the query tile
+      mbar_init(&sm.p_full[q], 4);
       mbar_init(&sm.o_done[q], 1);
       mbar_init(&sm.drain[q], 1);
-      mbar_init(&sm.xbar[q][0], 8);
-      mbar_init(&sm.xbar[q][1], 8);
-      mbar_init(&sm.lbar[q], 8);
     }
     sm.abort = 0;
     fence_barrier_init();
@@ -184,6 +167,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  if (warp >= kProducerWarp) {
+  regs_dealloc<kRegsAux>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA warp
     if (lane == 0) {
@@ -337,16 +322,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         if (lane == 0) mbar_arrive(&sm.v_ready[s]);
       }
     }
+  }
   } else {
+    regs_alloc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
-    const int q = warp >> 3;                       // query tile of the pair
-    const int hf = (warp >> 2) & 1;                // column half [64hf, 64hf + 64)
+    const int q = warp >> 2;                       // query tile of the pair
     const int r = ((warp & 3) << 5) + lane;        // row within the tile = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
-    const uint32_t t_s = tmem + lane_base + col_s(q) + 64 * hf;
-    const uint32_t t_p = tmem + lane_base + col_p(q) + 32 * hf;
-    const uint32_t t_o = tmem + lane_base + col_o(q) + 32 * hf;
-    uint32_t s_cnt = 0, o_cnt = 0, x_cnt = 0, l_cnt = 0;
+    const uint32_t t_s = tmem + lane_base + col_s(q);
+    const uint32_t t_p = tmem + lane_base + col_p(q);
+    const uint32_t t_o = tmem + lane_base + col_o(q);
+    uint32_t s_cnt = 0, o_cnt = 0;
     // The finished item whose O still sits in tensor memory. It is read out
     // while the next item's first tile is processed, just before that tile's
     // P goes to tensor memory (the next P V product then overwrites O); the
@@ -362,11 +348,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
       if (q == 1 && !it.has1) continue;
       const int i = it.i0 + q;
       const int row = i * kBlockM + r;
-      // Running max m (raw logit units, as read from S) and this half's running
-      // sum l of 2^(s*c - m*c), c = scale*log2(e). m is only raised when the
-      // row max grows by more than kRescaleLog2 in log2 units; until then P and
-      // l keep using the stale m, which stays exact because O / l uses the
-      // same m. Both halves of a row always hold the same m.
+      // Running max m (raw logit units, as read from S) and running sum l of
+      // 2^(s*c - m*c), c = scale*log2(e). m is only raised when the row max
+      // grows by more than kRescaleLog2 in log2 units; until then P and l keep
+      // using the stale m, which stays exact because O / l uses the same m.
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j <= i; ++j) {
         ok = mbar_wait(&sm.s_full[q], s_cnt & 1, kSiteFwdSoftmax, abort);
@@ -374,58 +359,45 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
-        float x[64];
+        float x[128];
         {
-          uint32_t u[64];
-          tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(u));
-          tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
-          tmem_wait_ld();
+          uint32_t* u = reinterpret_cast<uint32_t*>(x);
 #pragma unroll
-          for (int e = 0; e < 64; ++e) x[e] = __uint_as_float(u[e]);
+          for (int c = 0; c < 4; ++c)
+            tmem_ld32(t_s + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(u + 32 * c));
+          tmem_wait_ld();
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_free[q]);
 
         if (j == i) {
-          const int lim = row - j * kBlockN - 64 * hf;  // columns c > lim are future keys
+          const int lim = row - j * kBlockN;  // columns c > lim are future keys
 #pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
+          for (int c = 0; c < 128; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
         }
-        // Partial row max: 8 independent chains of 3-input max.
+        // Row max: 8 independent chains of 3-input max.
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = fmax3(x[e], x[8 + e], x[16 + e]);
 #pragma unroll
-        for (int c = 24; c < 56; c += 16) {
+        for (int c = 24; c < 120; c += 16) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], x[c + e], x[c + 8 + e]);
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[56 + e]);
-        float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                         fmaxf(mx8[6], mx8[7]));
-        // Exchange with the other half of the row.
-        {
-          const int buf = x_cnt & 1;
-          sm.xmax[q][buf][hf][r] = mx;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.xbar[q][buf]);
-          ok = mbar_wait(&sm.xbar[q][buf], (x_cnt >> 1) & 1, kSiteFwdSoftmax, abort);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          ++x_cnt;
-          mx = fmaxf(mx, sm.xmax[q][buf][hf ^ 1][r]);
-        }
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[120 + e]);
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
         const bool grow = (mx - m) * sh.scale_log2 > kRescaleLog2;  // always true on j == 0
         const float m_new = grow ? mx : m;
         const float alpha = grow ? ex2((m - m_new) * sh.scale_log2) : 1.f;
         const float neg_mc = -m_new * sh.scale_log2;
-        // p = 2^(s*c - m*c), partial row sum, and fp16 packing of P in one pass.
-        uint32_t pk[32];
+        // p = 2^(s*c - m*c), row sum, and fp16 packing of P in one pass.
+        uint32_t pk[64];
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
+        for (int c2 = 0; c2 < 64; ++c2) {
           float y0, y1;
           fma2(x[2 * c2], x[2 * c2 + 1], sh.scale_log2, neg_mc, y0, y1);
           const float p0 = ex2(y0), p1 = ex2(y1);
@@ -445,31 +417,35 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
           if (!ok) break;
           ++o_cnt;
           tc_fence_after();
-          if (!flush && __any_sync(0xffffffffu, grow)) {
-            uint32_t oo[32];
-            tmem_ld32(t_o, oo);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) oo[e] = __float_as_uint(__uint_as_float(oo[e]) * alpha);
-            tmem_st32(t_o, oo);
-            tmem_wait_st();
-          }
         }
-        tmem_st32(t_p, pk);
-        tmem_wait_st();
+        tmem_st32(t_p, *reinterpret_cast<uint32_t(*)[32]>(pk));
+        tmem_st32(t_p + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
         if (flush) {
           // The finished item's O is read before this tile's P V product (which
           // starts only after the arrival below) overwrites it.
-          uint32_t o[32];
-          tmem_ld32(t_o, o);
+          uint32_t o[64];
+          tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(o));
+          tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
           tmem_wait_ld();
+          tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.p_full[q]);
-          ok = finish_row(sm, q, hf, r, lane, l_cnt, abort, o, p_b, p_h, p_row, p_m, p_l, out, lse, sh);
-          if (!ok) break;
+          store_row(o, p_b, p_h, p_row, p_m, p_l, out, lse, sh);
           pending = false;
         } else {
+          if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              uint32_t oo[32];
+              tmem_ld32(t_o + 32 * c, oo);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) oo[e] = __float_as_uint(__uint_as_float(oo[e]) * alpha);
+              tmem_st32(t_o + 32 * c, oo);
+            }
+          }
+          tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.p_full[q]);
@@ -489,11 +465,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
       if (ok) {
         ++o_cnt;
         tc_fence_after();
-        uint32_t o[32];
-        tmem_ld32(t_o, o);
+        uint32_t o[64];
+        tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(o));
+        tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
         tmem_wait_ld();
         tc_fence_before();
-        finish_row(sm, q, hf, r, lane, l_cnt, abort, o, p_b, p_h, p_row, p_m, p_l, out, lse, sh);
+        store_row(o, p_b, p_h, p_row, p_m, p_l, out, lse, sh);
       }
     }
   }

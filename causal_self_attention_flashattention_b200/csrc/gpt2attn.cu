@@ -58,6 +58,13 @@ const DeviceInfo* device_info() {
   if (cudaFuncSetAttribute(ga::fwd::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(ga::fwd::kSmemBytes)) != cudaSuccess)
     return nullptr;
+  // The forward kernel's setmaxnreg split (warpgroup budgets that add up to the
+  // block's allocation) is only safe if it launches with the register count
+  // the split was sized for.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel) != cudaSuccess ||
+      fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
+    return nullptr;
 
   if (cudaFuncSetAttribute(ga::bwd::dkdv::attn_bwd_dkdv_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
