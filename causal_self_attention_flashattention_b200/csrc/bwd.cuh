@@ -84,43 +84,40 @@ constexpr float kLog2e = 1.4426950408889634f;
 // dK, dV: one CTA per key tile
 // ===========================================================================
 // Per query tile i >= j (all in the transposed frame, rows = keys):
-//   S^T  = K_j Q_i^T     (M128 N128 K64, both operands K-major)
-//   dP^T = V_j dO_i^T    (same)
-//   P^T  = exp2(S^T * scale*log2e - lse_i*log2e), zero where key > query
-//   dS^T = P^T o (dP^T - Delta_i)
+//   S'^T  = K_j Q_i^T - lse_i/scale   (M128 N128, K = 64 + one extra K16 step)
+//   dP'^T = V_j dO_i^T - Delta_i      (same)
+//   P^T   = exp2(S'^T * scale*log2e), zero where key > query
+//   dS^T  = P^T o dP'^T
+// The extra K step multiplies a constant tile A_ext (rows of ones in the
+// columns that pick a term) with a per-query tile B_ext holding -lse/scale and
+// -Delta, each split into three bf16 terms whose sum is exact to ~2^-24
+// relative. The per-query constants thus never pass through the elementwise
+// warps, which would otherwise broadcast them from shared memory while the
+// S/dP products saturate it.
 //   dV  += P^T dO_i      (A = P^T from tensor memory, B = dO_i MN-major)
 //   dK  += dS^T Q_i      (A = dS^T from tensor memory, B = Q_i MN-major)
 // Tensor memory: S^T [0,128), dP^T [128,256), P^T [256,320), dS^T [320,384)
 // (bf16 pairs), dV [384,448), dK [448,512).
-// 16 columns of one dK/dV tile row: P^T = 2^(S^T c - lse c) (zero where the
-// key r comes after query c0 + e when kMasked), dS^T = P^T (dP^T - Delta),
-// both packed to bf16 pairs.
+// 16 columns of one dK/dV tile row. The accumulators already hold
+// S^T - lse/scale and dP^T - Delta (one extra K step of each product adds the
+// per-query constants), so P^T = 2^(c x) (zero where the key r comes after
+// query c0 + e when kMasked) and dS^T = P^T o dP'^T, both packed to bf16 pairs.
 template <bool kMasked>
 __device__ __forceinline__ void dkdv_chunk(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
-                                           const float* nl, const float* nd, float sc, int c0,
-                                           int r, uint32_t (&pp)[8], uint32_t (&dd)[8]) {
+                                           float sc, int c0, int r, uint32_t (&pp)[8],
+                                           uint32_t (&dd)[8]) {
 #pragma unroll
-  for (int e4 = 0; e4 < 4; ++e4) {
-    const float4 L = reinterpret_cast<const float4*>(nl)[e4];
-    const float4 Dl = reinterpret_cast<const float4*>(nd)[e4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = 4 * e4 + 2 * h;
-      float x0, x1, t0, t1, d0, d1;
-      fma2v(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sc, sc, h ? L.z : L.x,
-            h ? L.w : L.y, x0, x1);
-      if (kMasked) {
-        if (c0 + c < r) x0 = -INFINITY;
-        if (c0 + c + 1 < r) x1 = -INFINITY;
-      }
-      const float p0 = ex2(x0), p1 = ex2(x1);
-      t0 = __uint_as_float(dv[c]);
-      t1 = __uint_as_float(dv[c + 1]);
-      add2(t0, t1, h ? Dl.z : Dl.x, h ? Dl.w : Dl.y);
-      mul2v(p0, p1, t0, t1, d0, d1);
-      pp[c >> 1] = pack_bf16(p0, p1);
-      dd[c >> 1] = pack_bf16(d0, d1);
+  for (int c = 0; c < 16; c += 2) {
+    float x0, x1, d0, d1;
+    mul2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sc, x0, x1);
+    if (kMasked) {
+      if (c0 + c < r) x0 = -INFINITY;
+      if (c0 + c + 1 < r) x1 = -INFINITY;
     }
+    const float p0 = ex2(x0), p1 = ex2(x1);
+    mul2v(p0, p1, __uint_as_float(dv[c]), __uint_as_float(dv[c + 1]), d0, d1);
+    pp[c >> 1] = pack_bf16(p0, p1);
+    dd[c >> 1] = pack_bf16(d0, d1);
   }
 }
 
@@ -188,13 +185,36 @@ __device__ __forceinline__ void store_dq_row(__nv_bfloat16* dqkv, const uint32_t
 
 namespace dkdv {
 
+constexpr uint32_t kExtBytes = 128 * 32;  // 128 rows x 16 bf16 (one K16 step)
+constexpr uint32_t kExtLbo = 128, kExtSbo = 256;
+
+// Byte offset of row `r`'s first 8 terms in an A_ext / B_ext tile.
+__device__ __forceinline__ uint32_t ext_row(int r) { return (r >> 3) * kExtSbo + (r & 7) * 16; }
+
+// v as three bf16 terms, each the nearest bf16 of what the previous ones
+// leave over: |v - (h1 + h2 + h3)| <= 2^-24 |v| (up to subnormals).
+__device__ __forceinline__ void split3_bf16(float v, __nv_bfloat16& h1, __nv_bfloat16& h2,
+                                            __nv_bfloat16& h3) {
+  h1 = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(h1);
+  h2 = __float2bfloat16_rn(r1);
+  h3 = __float2bfloat16_rn(r1 - __bfloat162float(h2));
+}
+
+__device__ __forceinline__ uint32_t bf16_pair(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+         (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
 struct alignas(1024) Smem {
   uint8_t k[2][kTileBytes];  // [item slot]
   uint8_t v[2][kTileBytes];
   uint8_t q[kStages][kTileBytes];
   uint8_t dout[kStages][kTileBytes];
-  float neg_lse2[kStages][kBlockM];  // -lse * log2(e) of the staged query tile
-  float neg_delta[kStages][kBlockM];  // -Delta of the staged query tile
+  // K-major, no swizzle: 8-row x 16-byte core matrices, 128 bytes apart along K
+  // (two per K16 step) and 256 bytes apart along the rows.
+  uint8_t ext_a[2][kExtBytes];        // [S, dP]: ones in terms 0-2 / 3-5 of every key row
+  uint8_t ext_b[kStages][kExtBytes];  // per query row: 3 terms of -lse/scale, 3 of -Delta
   uint64_t kv_full[2], kv_empty[2];
   uint64_t in_full[kStages], in_empty[kStages];
   uint64_t sdp_full, sdp_free, ds_full, pds_free;
@@ -203,6 +223,7 @@ struct alignas(1024) Smem {
   int abort;
 };
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+static_assert(kSmemBytes <= 232448, "dK/dV shared memory exceeds the 227 KiB per-block limit");
 
 __device__ __forceinline__ void decode(int k, const AttnShape& sh, int& b, int& h, int& j) {
   const int bh_count = sh.B * sh.H;
@@ -246,6 +267,19 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  // A_ext rows pick terms 0-2 (S) or 3-5 (dP) of B_ext; B_ext's second core
+  // matrix along K (terms 8-15) stays zero. Written through the generic proxy,
+  // so every writer fences before the tensor core may read them.
+  for (int idx = threadIdx.x; idx < 2 * kBlockN; idx += kThreads) {
+    const int which = idx / kBlockN, rr = idx % kBlockN;
+    uint4* a = reinterpret_cast<uint4*>(sm.ext_a[which] + ext_row(rr));
+    a[0] = which == 0 ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u)
+                      : make_uint4(0u, 0x3F800000u, 0x3F803F80u, 0u);
+    a[kExtLbo / 16] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  for (int idx = threadIdx.x; idx < kStages * static_cast<int>(kExtBytes / 16); idx += kThreads)
+    reinterpret_cast<uint4*>(&sm.ext_b[0][0])[idx] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&map_qkv);
     tma_prefetch_desc(&map_do);
@@ -260,8 +294,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
   const uint32_t tmem = sm.tmem_base;
 
   if (warp == kProducerWarp) {
-    // Lane 0 waits and issues the TMA copies; all 32 lanes stage the 128 lse
-    // (base 2) and Delta values of each query tile next to its Q and dO tiles.
+    // Lane 0 waits and issues the TMA copies; all 32 lanes write the query
+    // tile's B_ext (-lse/scale and -Delta as bf16 terms) next to its Q and dO.
+    const float inv_scale = 1.f / sh.scale;
     uint32_t in_it = 0, it_cnt = 0;
     bool ok = true;
     for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
@@ -292,11 +327,17 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
           const int c = lane + 32 * e;
           const int qrow = i * kBlockM + c;
           const bool valid = qrow < sh.T;
-          // Stored negated, so each becomes an addend of a fused multiply-add.
-          // Rows past T get -lse = -inf, so their P is exactly 0.
-          sm.neg_lse2[s][c] = valid ? -lse[row_base + qrow] * kLog2e : -INFINITY;
-          sm.neg_delta[s][c] = valid ? -delta[row_base + qrow] : 0.f;
+          // Rows past T get -1e30 (finite, so 0 x term stays 0 in the other
+          // product): their P underflows to exactly 0.
+          const float vl = valid ? -lse[row_base + qrow] * inv_scale : -1e30f;
+          const float vd = valid ? -delta[row_base + qrow] : 0.f;
+          __nv_bfloat16 l1, l2, l3, d1, d2, d3;
+          split3_bf16(vl, l1, l2, l3);
+          split3_bf16(vd, d1, d2, d3);
+          *reinterpret_cast<uint4*>(sm.ext_b[s] + ext_row(c)) =
+              make_uint4(bf16_pair(l1, l2), bf16_pair(l3, d1), bf16_pair(d2, d3), 0u);
         }
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive_expect_tx(&sm.in_full[s], 2 * kTileBytes);
@@ -316,9 +357,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    // S^T = K_j Q_i^T and dP^T = V_j dO_i^T for every query tile i >= j.
+    // S'^T and dP'^T (with the extra K step) for every query tile i >= j.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      const uint64_t aext_s = smem_desc_noswizzle(smem_u32(sm.ext_a[0]), kExtLbo, kExtSbo);
+      const uint64_t aext_dp = smem_desc_noswizzle(smem_u32(sm.ext_a[1]), kExtLbo, kExtSbo);
       const uint32_t t_s = tmem + 0, t_dp = tmem + 128;
       uint32_t in_it = 0, it_cnt = 0, sdp_cnt = 0;
       bool ok = true;
@@ -341,12 +384,15 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
           tc_fence_after();
           const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.q[s]), 16, 1024);
           const uint64_t odesc = smem_desc_sw128(smem_u32(sm.dout[s]), 16, 1024);
+          const uint64_t bext = smem_desc_noswizzle(smem_u32(sm.ext_b[s]), kExtLbo, kExtSbo);
           mma_ss(t_s, kdesc, qdesc, idesc_s, 0u);
 #pragma unroll
           for (int kk = 1; kk < kD / 16; ++kk) mma_ss(t_s, kdesc + 2 * kk, qdesc + 2 * kk, idesc_s, 1u);
+          mma_ss(t_s, aext_s, bext, idesc_s, 1u);
           mma_ss(t_dp, vdesc, odesc, idesc_s, 0u);
 #pragma unroll
           for (int kk = 1; kk < kD / 16; ++kk) mma_ss(t_dp, vdesc + 2 * kk, odesc + 2 * kk, idesc_s, 1u);
+          mma_ss(t_dp, aext_dp, bext, idesc_s, 1u);
           mma_commit(&sm.sdp_full);
           ++sdp_cnt;
         }
@@ -428,16 +474,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
       int b, h, j;
       decode(k, sh, b, h, j);
       for (int i = j; i < n_qt; ++i, ++in_it) {
-        // The stage's in_full phase (already complete: the MMA warp waited on
-        // it) makes the producer's lse/Delta stores visible to this thread.
-        ok = mbar_wait(&sm.in_full[in_it % kStages], (in_it / kStages) & 1, kSiteDkvSoftmax, abort);
-        ok = ok && mbar_wait(&sm.sdp_full, sdp_cnt & 1, kSiteDkvSoftmax, abort);
+        ok = mbar_wait(&sm.sdp_full, sdp_cnt & 1, kSiteDkvSoftmax, abort);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++sdp_cnt;
         tc_fence_after();
-        const float* nl = sm.neg_lse2[in_it % kStages] + 32 * g;
-        const float* nd = sm.neg_delta[in_it % kStages] + 32 * g;
         // Both 16-column halves are computed into registers before waiting for
         // the previous dV/dK products to release P^T and dS^T, so that wait
         // overlaps all of this tile's elementwise work.
@@ -459,9 +500,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
           // On the diagonal tile, a chunk needs the mask if one of its columns
           // lies before one of this warp's rows (key after query).
           if (i == j && c0 < r_lo + 31)
-            dkdv_chunk<true>(sv, dv, nl + 16 * half, nd + 16 * half, sc, c0, r, pph, ddh);
+            dkdv_chunk<true>(sv, dv, sc, c0, r, pph, ddh);
           else
-            dkdv_chunk<false>(sv, dv, nl + 16 * half, nd + 16 * half, sc, c0, r, pph, ddh);
+            dkdv_chunk<false>(sv, dv, sc, c0, r, pph, ddh);
         }
         const bool flush = (i == j) && pending;
         if (i > j || flush) {
