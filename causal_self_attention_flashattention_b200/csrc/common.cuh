@@ -24,7 +24,7 @@ enum WaitSite : uint32_t {
   kSiteFwdMma = 0x102,
   kSiteFwdSoftmax = 0x103,
   kSiteFwdConvert = 0x104,
-  kFwdValueRange = 0x1F0,  // a V entry outside the fp16 range (|v| > 65504)
+  kFwdValueRange = 0x1F0,  // a V entry outside the fp16 range (|v| > 65504, inf, NaN)
   kSiteDqProducer = 0x201,
   kSiteDqMma = 0x202,
   kSiteDqSoftmax = 0x203,

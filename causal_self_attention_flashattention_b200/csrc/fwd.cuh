@@ -28,7 +28,8 @@
 //     [0, 1] keeps 11 significant bits instead of 8, which matters on peaked
 //     rows where one probability near 1 multiplies a large v. Every bf16 value
 //     with |v| <= 65504 converts exactly (tiny ones to fp16 subnormals, within
-//     3e-8); a finite |v| above 65504 is reported in the status word.
+//     3e-8); a v that is not finite with |v| <= 65504 is reported in the
+//     status word.
 //
 // Tensor memory (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256),
 // P_0 [256,320), P_1 [320,384) (fp16 pairs), O_0 [384,448), O_1 [448,512).
@@ -61,6 +62,8 @@ static_assert(kProducerWarp == 8 && kConvertWarp == 11, "warps 8-11 form the aux
 // The running max is raised only when a row's max grows by more than this many
 // powers of two; until then P may reach 2^8 (well inside fp16).
 constexpr float kRescaleLog2 = 8.f;
+// One pair in kPolyEvery is exponentiated with the FMA-pipe polynomial.
+constexpr int kPolyEvery = 4;
 constexpr uint32_t kTmemCols = 512;
 
 __device__ __forceinline__ uint32_t col_s(int q) { return q * 128; }
@@ -300,22 +303,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         uint4* tile = reinterpret_cast<uint4*>(sm.v[s]);
-        bool bad = false;
+        // Running max of |v| over the converted fp16 values: a bf16 beyond
+        // fp16's range rounds to inf, so inf or NaN here flags the tile.
+        uint32_t mag = 0;
 #pragma unroll 4
         for (int c = lane; c < kTileBytes / 16; c += 32) {
           uint4 w = tile[c];
           uint32_t* u = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            bad |= bf16x2_out_of_f16_range(u[e]) != 0;
             // bf16 -> fp32 is exact (a shift); fp32 -> fp16 rounds to nearest,
             // exact for every bf16 value with |v| <= 65504 except fp16
             // subnormals (|v| < 6.1e-5, within 3e-8).
             u[e] = pack_f16(__uint_as_float(u[e] << 16), __uint_as_float(u[e] & 0xFFFF0000u));
+            mag = max_abs_f16x2(mag, u[e]);
           }
           tile[c] = w;
         }
-        if (bad) record_failure(kFwdValueRange);
+        if ((mag & 0x7FFFu) >= kF16InfBits || ((mag >> 16) & 0x7FFFu) >= kF16InfBits)
+          record_failure(kFwdValueRange);
         // Generic-proxy stores must be visible to the tensor core (async proxy).
         fence_proxy_async_smem();
         __syncwarp();
@@ -393,14 +399,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         const float m_new = grow ? mx : m;
         const float alpha = grow ? ex2((m - m_new) * sh.scale_log2) : 1.f;
         const float neg_mc = -m_new * sh.scale_log2;
-        // p = 2^(s*c - m*c), row sum, and fp16 packing of P in one pass.
+        // p = 2^(s*c - m*c), row sum, and fp16 packing of P in one pass. Every
+        // kPolyEvery-th pair is exponentiated on the FMA pipe (exp2_poly2), the
+        // rest on the exp unit, whose 16/clk rate bounds this loop otherwise.
         uint32_t pk[64];
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c2 = 0; c2 < 64; ++c2) {
-          float y0, y1;
+          float y0, y1, p0, p1;
           fma2(x[2 * c2], x[2 * c2 + 1], sh.scale_log2, neg_mc, y0, y1);
-          const float p0 = ex2(y0), p1 = ex2(y1);
+          if (c2 % kPolyEvery == kPolyEvery - 1) {
+            exp2_poly2(y0, y1, p0, p1);
+          } else {
+            p0 = ex2(y0);
+            p1 = ex2(y1);
+          }
           add2(sa[c2 & 3], sb[c2 & 3], p0, p1);
           pk[c2] = pack_f16_nonneg(p0, p1);
         }

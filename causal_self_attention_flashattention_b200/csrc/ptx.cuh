@@ -408,6 +408,38 @@ __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
       : "f"(b0), "f"(b1));
 }
 
+// 2^y for a pair of floats on the FMA/ALU pipes instead of the 16/clk exp
+// unit. y = n + f with n = rint(y) (adding 1.5 * 2^23 rounds y to an integer
+// that lands in the low mantissa bits), 2^f from a cubic, and n added to the
+// exponent field. The cubic was fitted to 2^f on [-1/2, 1/2] by least squares
+// on Chebyshev nodes, reweighted toward equal ripple (Lawson's iteration); its
+// largest relative error there is 7.5e-5. y is clamped to >= -125 first, so
+// the exponent never wraps: -inf and very negative y give a value below
+// 2^-125 instead of 0.
+constexpr float kExp2Poly0 = 0.9999280571937561f;
+constexpr float kExp2Poly1 = 0.6932609677314758f;
+constexpr float kExp2Poly2 = 0.2426111251115799f;
+constexpr float kExp2Poly3 = 0.0551716648042202f;
+
+__device__ __forceinline__ void exp2_poly2(float y0, float y1, float& p0, float& p1) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  const float a0 = fmaxf(y0, -125.f), a1 = fmaxf(y1, -125.f);
+  float t0 = a0, t1 = a1;
+  add2(t0, t1, kRound, kRound);
+  float n0 = t0, n1 = t1;
+  add2(n0, n1, -kRound, -kRound);
+  float f0, f1;
+  fma2v(n0, n1, -1.f, -1.f, a0, a1, f0, f1);  // f = a - n, in [-1/2, 1/2]
+  float q0, q1;
+  fma2(f0, f1, kExp2Poly3, kExp2Poly2, q0, q1);
+  fma2v(q0, q1, f0, f1, kExp2Poly1, kExp2Poly1, q0, q1);
+  fma2v(q0, q1, f0, f1, kExp2Poly0, kExp2Poly0, q0, q1);
+  // bits(t) << 23 == n << 23 (mod 2^32): the rounding constant's own bits
+  // shift out.
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
@@ -428,30 +460,16 @@ __device__ __forceinline__ uint32_t pack_f16_nonneg(float lo, float hi) {
   return (b0 >> 13) | ((b1 << 3) & 0xFFFF0000u);
 }
 
-// Two bf16 values (one 32-bit word) to two fp16 values. Exact for
-// |v| <= 65504 (subnormal results round half up); larger finite magnitudes
-// are not representable and must be caught with bf16x2_out_of_f16_range.
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
-  float m0, m1;
-  mul2(__uint_as_float((w << 16) & 0x7FFF0000u), __uint_as_float(w & 0x7FFF0000u),
-       kF32ToF16Scale, m0, m1);
-  const uint32_t b0 = __float_as_uint(m0) + 0x1000u;
-  const uint32_t b1 = __float_as_uint(m1) + 0x1000u;
-  return (w & 0x80008000u) | (b0 >> 13) | ((b1 << 3) & 0x7FFF0000u);
+// Per fp16 half: the larger magnitude of a and b (its sign is the xor of the
+// signs, which callers ignore); a NaN in either input gives NaN.
+__device__ __forceinline__ uint32_t max_abs_f16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
-// Nonzero iff a half of the bf16x2 word is finite with |v| >= 65536 (the
-// first bf16 magnitude above 65504).
-__device__ __forceinline__ uint32_t bf16x2_out_of_f16_range(uint32_t w) {
-  const uint32_t t = w & 0x7FFF7FFFu;
-  return ((t + 0x38803880u) & ~(t + 0x00800080u)) & 0x80008000u;
-}
-
-// Two floats to bf16x2, rounding half away from zero on the dropped bits
-// (differs from round-to-nearest-even only on exact ties).
-__device__ __forceinline__ uint32_t pack_bf16_fast(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
+// Magnitude bits of an fp16 at or above this: inf or NaN.
+constexpr uint32_t kF16InfBits = 0x7C00u;
 
 // Warpgroup-wide register budget changes (all four warps of a warpgroup
 // execute the same one). The budgets of all warpgroups must add up to no more

@@ -59,7 +59,7 @@ typedef enum {
   GA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the query result */
   GA_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed */
   GA_ERR_TIMEOUT = 6,     /* a device-side wait gave up (see gpt2_attn_last_device_status) */
-  GA_ERR_RANGE = 7        /* the forward met a finite v entry with |v| > 65504 (fp16 range) */
+  GA_ERR_RANGE = 7        /* the forward met a v entry outside the fp16 range (|v| > 65504, inf or NaN) */
 } ga_status;
 
 /*
@@ -73,9 +73,9 @@ typedef enum {
  * registers, key tiles above the diagonal are skipped, and lse is written
  * per query row. S = Q K^T multiplies bf16 operands. O += P V multiplies
  * fp16 operands: P keeps 11 significant bits, and each bf16 v converts to
- * fp16 exactly when |v| <= 65504. A finite |v| above that is reported as
- * GA_ERR_RANGE by gpt2_attn_last_device_status; the outputs of that call are
- * then undefined.
+ * fp16 exactly when |v| <= 65504. A v entry with |v| above that, or an inf or
+ * NaN, is reported as GA_ERR_RANGE by gpt2_attn_last_device_status; the
+ * outputs of that call are then undefined.
  */
 ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse,
                         int B, int T, int H, int D, float scale,

@@ -232,6 +232,30 @@ def test_autograd_wrapper(ops):
     assert rel_fro(x.grad.cpu().double().numpy(), dqkv_o) <= GRAD_TOL
 
 
+@pytest.mark.parametrize("v_val,flagged", [
+    (65280.0, False),         # the largest bf16 below fp16's 65504: converts exactly
+    (-65280.0, False),
+    (65536.0, True),          # the next bf16 up has no fp16 counterpart
+    (-1.0e6, True),
+    (float("inf"), True),
+    (float("nan"), True),
+])
+def test_v_outside_fp16_range_is_reported(ops, v_val, flagged):
+    """The forward's P.V product runs in fp16, so a V entry fp16 cannot hold is
+    reported as GA_ERR_RANGE (and the word is cleared by reading it)."""
+    qkv_bf, _ = make_inputs(1, 300, 2, 64, seed=12)
+    qkv_bf[0, 257, 2, 1, 5] = v_val          # one V entry in the last, ragged key tile
+    qkv = qkv_bf.cuda()
+    out, lse = ops.attn_fwd(qkv)
+    st, word = ops.last_device_status()
+    if flagged:
+        assert st == ops.GA_ERR_RANGE and word != 0, (st, hex(word))
+    else:
+        assert st == ops.GA_OK and word == 0, (st, hex(word))
+        assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    assert ops.last_device_status() == (ops.GA_OK, 0)
+
+
 def test_status_word_clean_after_runs(ops):
     st, word = ops.last_device_status()
     assert st == ops.GA_OK and word == 0
