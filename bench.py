@@ -294,8 +294,8 @@ def run_ours(args, wl):
         if ev is not None:
             ev[0].record(stream)
         ops.attn_fwd(s["qkv"], scale, out=s["out"], lse=s["lse"], stream=stream)
-        ops.attn_bwd_steps(s["qkv"], s["out"], s["dout"], s["lse"], s["delta"], s["dqkv"], scale,
-                           stream=stream, events=None if ev is None else ev[1:])
+        ops.attn_bwd_split_steps(s["qkv"], s["out"], s["dout"], s["lse"], s["delta"], s["dqkv"],
+                                 scale, stream=stream, events=None if ev is None else ev[1:])
 
     for i in range(args.warmup):
         step(sets[i % n_sets])

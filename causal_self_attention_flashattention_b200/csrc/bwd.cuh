@@ -29,9 +29,14 @@ namespace bwd {
 // ===========================================================================
 // Eight lanes per (b, t, h) row of 64 bf16: each lane loads 16 bytes of both
 // tensors, and three shuffles finish the dot product.
+// Also zeroes `n_counters` words at `counters` (the fused backward's dQ
+// ordering counters; none for the split backward).
 __global__ void __launch_bounds__(256)
 attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
-                    float* __restrict__ delta, const AttnShape sh) {
+                    float* __restrict__ delta, uint32_t* __restrict__ counters, int n_counters,
+                    const AttnShape sh) {
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < n_counters; c += gridDim.x * blockDim.x)
+    counters[c] = 0u;
   const long long rows = static_cast<long long>(sh.B) * sh.T * sh.H;
   const int sub = threadIdx.x & 7;
   // The 8 lanes of one row always take the same branch, so the shuffles only

@@ -31,6 +31,10 @@ enum WaitSite : uint32_t {
   kSiteDkvProducer = 0x301,
   kSiteDkvMma = 0x302,
   kSiteDkvSoftmax = 0x303,
+  kSiteFusedProducer = 0x401,
+  kSiteFusedMma = 0x402,
+  kSiteFusedSoftmax = 0x403,
+  kSiteFusedDq = 0x404,  // waiting for earlier key tiles' dQ sums
 };
 
 struct AttnShape {

@@ -20,6 +20,7 @@
 #include "ptx.cuh"
 #include "fwd.cuh"
 #include "bwd.cuh"
+#include "bwd_fused.cuh"
 
 namespace {
 
@@ -70,6 +71,10 @@ const DeviceInfo* device_info() {
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(ga::bwd::dkdv::kSmemBytes)) != cudaSuccess)
     return nullptr;
+  if (cudaFuncSetAttribute(ga::bwd::fused::attn_bwd_fused_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::bwd::fused::kSmemBytes)) != cudaSuccess)
+    return nullptr;
   if (cudaFuncSetAttribute(ga::bwd::dq::attn_bwd_dq_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(ga::bwd::dq::kSmemBytes)) != cudaSuccess)
@@ -118,12 +123,12 @@ ga::AttnShape make_shape(int B, int T, int H, float scale) {
   return sh;
 }
 
+int grid_for(int items, int num_sms) { return items < num_sms ? items : num_sms; }
+
 size_t delta_bytes(int B, int T, int H) {
   const size_t n = static_cast<size_t>(B) * H * T * sizeof(float);
   return (n + 255) & ~static_cast<size_t>(255);
 }
-
-int grid_for(int items, int num_sms) { return items < num_sms ? items : num_sms; }
 
 }  // namespace
 
@@ -158,12 +163,18 @@ ga_status gpt2_attn_bwd_workspace_size(int B, int T, int H, int D, size_t* bytes
   return GA_OK;
 }
 
-ga_status gpt2_attn_bwd_preprocess(const void* out, const void* dout, float* delta, int B,
-                                   int T, int H, int D, gpt2attn_stream_t stream) {
-  if (out == nullptr || dout == nullptr || delta == nullptr) return GA_ERR_INVALID_ARG;
+ga_status gpt2_attn_bwd_fused_workspace_size(int B, int T, int H, int D, size_t* bytes) {
+  if (bytes == nullptr) return GA_ERR_INVALID_ARG;
   const ga_status st = check_shape(B, T, H, D);
   if (st != GA_OK) return st;
-  if (!aligned16(out) || !aligned16(dout) || !aligned16(delta)) return GA_ERR_ALIGNMENT;
+  *bytes = ga::bwd::fused::ws_bytes(B, T, H);
+  return GA_OK;
+}
+
+namespace {
+
+ga_status launch_pre(const void* out, const void* dout, float* delta, uint32_t* counters,
+                     int n_counters, int B, int T, int H, gpt2attn_stream_t stream) {
   const DeviceInfo* info = device_info();
   if (info == nullptr) return GA_ERR_CUDA;
   const ga::AttnShape sh = make_shape(B, T, H, 1.f);
@@ -172,8 +183,35 @@ ga_status gpt2_attn_bwd_preprocess(const void* out, const void* dout, float* del
   const long long cap = 16LL * info->num_sms;
   const int blocks = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
   ga::bwd::attn_bwd_pre_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta, sh);
+      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta,
+      counters, n_counters, sh);
   return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+}
+
+}  // namespace
+
+ga_status gpt2_attn_bwd_preprocess(const void* out, const void* dout, float* delta, int B,
+                                   int T, int H, int D, gpt2attn_stream_t stream) {
+  if (out == nullptr || dout == nullptr || delta == nullptr) return GA_ERR_INVALID_ARG;
+  const ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(delta)) return GA_ERR_ALIGNMENT;
+  return launch_pre(out, dout, delta, nullptr, 0, B, T, H, stream);
+}
+
+ga_status gpt2_attn_bwd_prepare(const void* out, const void* dout, void* workspace,
+                                size_t workspace_bytes, int B, int T, int H, int D,
+                                gpt2attn_stream_t stream) {
+  if (out == nullptr || dout == nullptr) return GA_ERR_INVALID_ARG;
+  const ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if (workspace == nullptr || workspace_bytes < ga::bwd::fused::ws_bytes(B, T, H))
+    return GA_ERR_WORKSPACE;
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(workspace)) return GA_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return launch_pre(out, dout, reinterpret_cast<float*>(ws),
+                    reinterpret_cast<uint32_t*>(ws + ga::bwd::fused::ws_cnt_offset(B, T, H)),
+                    B * H * ga::ceil_div(T, ga::kBlockM), B, T, H, stream);
 }
 
 namespace {
@@ -227,6 +265,26 @@ ga_status gpt2_attn_bwd_dq(const void* qkv, const void* dout, const float* lse,
   ga::bwd::dq::attn_bwd_dq_kernel<<<L.grid, ga::bwd::kThreads, ga::bwd::dq::kSmemBytes,
                                     reinterpret_cast<cudaStream_t>(stream)>>>(
       L.map_qkv, L.map_do, lse, delta, static_cast<__nv_bfloat16*>(dqkv), L.sh);
+  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+}
+
+ga_status gpt2_attn_bwd_fused(const void* qkv, const void* dout, const float* lse,
+                              void* workspace, size_t workspace_bytes, void* dqkv, int B, int T,
+                              int H, int D, float scale, gpt2attn_stream_t stream) {
+  if (workspace == nullptr) return GA_ERR_WORKSPACE;
+  BwdLaunch L;
+  const ga_status st = prepare_bwd(qkv, dout, lse, static_cast<const float*>(workspace), dqkv, B,
+                                   T, H, D, scale, &L);
+  if (st != GA_OK) return st;
+  if (workspace_bytes < ga::bwd::fused::ws_bytes(B, T, H)) return GA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  ga::bwd::fused::attn_bwd_fused_kernel<<<L.grid, ga::bwd::fused::kFusedThreads,
+                                          ga::bwd::fused::kSmemBytes,
+                                          reinterpret_cast<cudaStream_t>(stream)>>>(
+      L.map_qkv, L.map_do, lse, reinterpret_cast<const float*>(ws),
+      reinterpret_cast<float*>(ws + ga::bwd::fused::ws_dq_offset(B, T, H)),
+      reinterpret_cast<uint32_t*>(ws + ga::bwd::fused::ws_cnt_offset(B, T, H)),
+      static_cast<__nv_bfloat16*>(dqkv), L.sh);
   return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
 }
 

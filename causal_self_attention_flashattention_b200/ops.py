@@ -38,6 +38,9 @@ EXPORTED_SYMBOLS = (
     "gpt2_attn_fwd",
     "gpt2_attn_bwd_workspace_size",
     "gpt2_attn_bwd",
+    "gpt2_attn_bwd_fused_workspace_size",
+    "gpt2_attn_bwd_prepare",
+    "gpt2_attn_bwd_fused",
     "gpt2_attn_bwd_preprocess",
     "gpt2_attn_bwd_dkdv",
     "gpt2_attn_bwd_dq",
@@ -57,6 +60,14 @@ _lib.gpt2_attn_bwd_workspace_size.restype = _i
 _lib.gpt2_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
                                _i, _i, _i, _i, _f, _vp]
 _lib.gpt2_attn_bwd.restype = _i
+_lib.gpt2_attn_bwd_fused_workspace_size.argtypes = [_i, _i, _i, _i,
+                                                   ctypes.POINTER(ctypes.c_size_t)]
+_lib.gpt2_attn_bwd_fused_workspace_size.restype = _i
+_lib.gpt2_attn_bwd_prepare.argtypes = [_vp, _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _vp]
+_lib.gpt2_attn_bwd_prepare.restype = _i
+_lib.gpt2_attn_bwd_fused.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_size_t, _vp,
+                                     _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_bwd_fused.restype = _i
 _lib.gpt2_attn_bwd_preprocess.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp]
 _lib.gpt2_attn_bwd_preprocess.restype = _i
 _lib.gpt2_attn_bwd_dkdv.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
@@ -155,7 +166,7 @@ def bwd_workspace_size(B: int, T: int, H: int, D: int) -> int:
 def attn_bwd(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor,
              scale: float | None = None, dqkv: torch.Tensor | None = None,
              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Causal attention backward: returns dqkv (B,T,3,H,D) bf16.
+    """Causal attention backward: returns dqkv (B,T,3,H,D) bf16 (bitwise deterministic).
 
     ``workspace`` (a uint8 CUDA tensor of at least ``bwd_workspace_size`` bytes)
     is allocated here when not given; after the call its first B*H*T fp32
@@ -170,27 +181,85 @@ def attn_bwd(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor, lse: torc
     if dqkv is None:
         dqkv = torch.empty_like(qkv)
     _expect(dqkv, "dqkv", (B, T, 3, H, D), torch.bfloat16)
-    need = bwd_workspace_size(B, T, H, D)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=qkv.device)
-    if not workspace.is_cuda or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous CUDA tensor")
-    ws_bytes = workspace.numel() * workspace.element_size()
+        workspace = torch.empty(bwd_workspace_size(B, T, H, D), dtype=torch.uint8,
+                                device=qkv.device)
+    ws, ws_bytes = _workspace(workspace)
     _check(_lib.gpt2_attn_bwd(qkv.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
-                              dqkv.data_ptr(), workspace.data_ptr(), ws_bytes, B, T, H, D,
+                              dqkv.data_ptr(), ws, ws_bytes, B, T, H, D,
                               scale, _stream_ptr(stream)), "gpt2_attn_bwd")
     return dqkv
 
 
-def attn_bwd_steps(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor,
-                   delta: torch.Tensor, dqkv: torch.Tensor, scale: float | None = None,
-                   stream=None, events=None) -> torch.Tensor:
-    """The backward as its three separate C-ABI steps (preprocess, dK/dV, dQ).
+def bwd_fused_workspace_size(B: int, T: int, H: int, D: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.gpt2_attn_bwd_fused_workspace_size(B, T, H, D, ctypes.byref(n)),
+           "gpt2_attn_bwd_fused_workspace_size")
+    return int(n.value)
+
+
+def _workspace(workspace: torch.Tensor):
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def attn_bwd_fused_steps(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+                         lse: torch.Tensor, workspace: torch.Tensor, dqkv: torch.Tensor,
+                         scale: float | None = None, stream=None, events=None) -> torch.Tensor:
+    """The fused backward as its two C-ABI steps (prepare, fused kernel).
+
+    ``workspace`` has at least ``bwd_fused_workspace_size`` bytes. Same dqkv as
+    ``attn_bwd`` up to fp32 summation order in dq. If ``events`` (three CUDA
+    events) is given, they are recorded on the stream before, between and
+    after the two launches, so each step can be timed on the device.
+    """
+    B, T, H, D = _dims(qkv)
+    _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
+    _expect(out, "out", (B, T, H, D), torch.bfloat16)
+    _expect(dout, "dout", (B, T, H, D), torch.bfloat16)
+    _expect(lse, "lse", (B, H, T), torch.float32)
+    _expect(dqkv, "dqkv", (B, T, 3, H, D), torch.bfloat16)
+    scale = default_scale(D) if scale is None else float(scale)
+    ws, ws_bytes = _workspace(workspace)
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    sp = _stream_ptr(stream)
+    if events is not None:
+        events[0].record(stream)
+    _check(_lib.gpt2_attn_bwd_prepare(out.data_ptr(), dout.data_ptr(), ws, ws_bytes,
+                                      B, T, H, D, sp), "gpt2_attn_bwd_prepare")
+    if events is not None:
+        events[1].record(stream)
+    _check(_lib.gpt2_attn_bwd_fused(qkv.data_ptr(), dout.data_ptr(), lse.data_ptr(), ws, ws_bytes,
+                                    dqkv.data_ptr(), B, T, H, D, scale, sp), "gpt2_attn_bwd_fused")
+    if events is not None:
+        events[2].record(stream)
+    return dqkv
+
+
+def attn_bwd_fused(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor,
+                   scale: float | None = None, dqkv: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The fused backward (gpt2_attn_bwd_prepare + gpt2_attn_bwd_fused)."""
+    B, T, H, D = _dims(qkv)
+    if dqkv is None:
+        dqkv = torch.empty_like(qkv)
+    if workspace is None:
+        workspace = torch.empty(bwd_fused_workspace_size(B, T, H, D), dtype=torch.uint8,
+                                device=qkv.device)
+    return attn_bwd_fused_steps(qkv, out, dout, lse, workspace, dqkv, scale, stream)
+
+
+def attn_bwd_split_steps(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+                         lse: torch.Tensor, delta: torch.Tensor, dqkv: torch.Tensor,
+                         scale: float | None = None, stream=None, events=None) -> torch.Tensor:
+    """``attn_bwd`` as its three C-ABI steps (preprocess, dK/dV, dQ).
 
     Same result as ``attn_bwd``. ``delta`` is a caller-owned fp32 (B,H,T)
-    tensor. If ``events`` (four CUDA events) is given, they are recorded on
-    the stream before, between and after the three launches, so each step can
-    be timed on the device.
+    tensor. If ``events`` (four CUDA events) is given, they are recorded on the
+    stream before, between and after the three launches, so each step can be
+    timed on the device.
     """
     B, T, H, D = _dims(qkv)
     _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)

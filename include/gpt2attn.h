@@ -82,8 +82,8 @@ ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse,
                         gpt2attn_stream_t stream);
 
 /*
- * Size in bytes of the workspace gpt2_attn_bwd needs for this shape.
- * Layout of the workspace: Delta, fp32 (B,H,T), at offset 0, where
+ * Size in bytes of the workspace gpt2_attn_bwd needs for this shape:
+ * Delta, fp32 (B,H,T), at offset 0, rounded up to 256 bytes, where
  * Delta[b,h,t] = sum_d dout[b,t,h,d] * out[b,t,h,d]. After a gpt2_attn_bwd
  * call it holds that call's Delta.
  */
@@ -97,9 +97,9 @@ ga_status gpt2_attn_bwd_workspace_size(int B, int T, int H, int D, size_t* bytes
  *   workspace [scratch] device, >= gpt2_attn_bwd_workspace_size bytes,
  *             16-byte aligned, owned by the caller, must not be shared by
  *             calls that run concurrently
- * Three launches on `stream`: Delta = rowsum(dout * out); dk and dv per key
- * tile, which recompute P from lse; dq per query tile, which recomputes P and
- * accumulates dq in tensor memory with no atomics. The result is bitwise
+ * Three launches on `stream` (the split backward below): Delta; dk and dv per
+ * key tile, which recompute P from lse; dq per query tile, which recomputes P
+ * and accumulates dq in tensor memory with no atomics. The result is bitwise
  * deterministic.
  */
 ga_status gpt2_attn_bwd(const void* qkv, const void* out, const void* dout,
@@ -132,6 +132,39 @@ ga_status gpt2_attn_bwd_dq(const void* qkv, const void* dout, const float* lse,
                            const float* delta, void* dqkv,
                            int B, int T, int H, int D, float scale,
                            gpt2attn_stream_t stream);
+
+/*
+ * The fused backward: the same dqkv from one pass over the causal tiles
+ * (S, P, dP, dS computed once per tile instead of twice), bitwise
+ * deterministic. On B200 at GPT-2 shapes it is slower than gpt2_attn_bwd:
+ * the ordered dq reduction across CTAs costs more than the recompute it
+ * saves. It needs a larger workspace, with n = ceil(T/128):
+ * 4*B*H*T + 4*B*H*(128n)*D + 4*B*H*n bytes, each part rounded up to 256.
+ * Layout, byte offsets:
+ *   0                          Delta fp32 (B,H,T)
+ *   align256(4*B*H*T)          dq partial sums, fp32, per 128-row query tile
+ *   + align256(4*B*H*128n*D)   dq ordering counters, uint32 (B,H,n)
+ *
+ * gpt2_attn_bwd_fused_workspace_size: that size.
+ * gpt2_attn_bwd_prepare: Delta into the workspace, and zeroes its counters.
+ *   GA_ERR_WORKSPACE if the workspace is missing or too small.
+ * gpt2_attn_bwd_fused: needs a workspace prepared by gpt2_attn_bwd_prepare
+ *   for the same out, dout and shape (earlier on the same stream). One CTA
+ *   per 128-key tile j recomputes P from lse for every query tile i >= j
+ *   (from the last to the diagonal one) and issues dV += P^T dO and
+ *   dK += dS^T Q (kept in tensor memory) and dQ_ij = dS K_j. Each dQ_ij is
+ *   added to the workspace's fp32 sum for query tile i in ascending j (key
+ *   tile j waits until tiles 0..j-1 have added); key tile i adds last and
+ *   writes dq = scale * sum as bf16. Writes all three dqkv slots.
+ */
+ga_status gpt2_attn_bwd_fused_workspace_size(int B, int T, int H, int D, size_t* bytes);
+ga_status gpt2_attn_bwd_prepare(const void* out, const void* dout, void* workspace,
+                                size_t workspace_bytes, int B, int T, int H, int D,
+                                gpt2attn_stream_t stream);
+ga_status gpt2_attn_bwd_fused(const void* qkv, const void* dout, const float* lse,
+                              void* workspace, size_t workspace_bytes, void* dqkv,
+                              int B, int T, int H, int D, float scale,
+                              gpt2attn_stream_t stream);
 
 /*
  * gpt2_attn_bwd without a workspace argument, for callers that cannot

@@ -94,9 +94,22 @@ def test_bwd_rejects(kw, status):
     assert bwd(**kw) == status
 
 
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
 def test_workspace_size():
+    # The split backward: Delta fp32 (B,H,T), rounded up to 256 bytes.
     assert ops.bwd_workspace_size(16, 1024, 12, 64) == 16 * 12 * 1024 * 4
-    assert ops.bwd_workspace_size(1, 5, 1, 64) == 256  # rounded up to 256 bytes
+    assert ops.bwd_workspace_size(1, 5, 1, 64) == 256
+    # The fused backward: Delta | dQ sums fp32 (B,H,128*ceil(T/128),D) |
+    # counters u32 (B,H,ceil(T/128)), each part rounded up to 256 bytes.
+    def layout(B, T, H):
+        n = -(-T // 128)
+        return (_align256(4 * B * H * T) + _align256(4 * B * H * 128 * n * 64)
+                + _align256(4 * B * H * n))
+    assert ops.bwd_fused_workspace_size(16, 1024, 12, 64) == layout(16, 1024, 12) == 51_124_224
+    assert ops.bwd_fused_workspace_size(1, 5, 1, 64) == layout(1, 5, 1) == 256 + 32768 + 256
     n = ctypes.c_size_t(0)
     assert ops.lib().gpt2_attn_bwd_workspace_size(1, 8, 1, 64, None) == ops.GA_ERR_INVALID_ARG
     assert ops.lib().gpt2_attn_bwd_workspace_size(1, 8, 1, 48, ctypes.byref(n)) == ops.GA_ERR_UNSUPPORTED

@@ -152,6 +152,58 @@ def test_full_size_workloads_sampled_heads(ops, name, heads):
     sampled_heads_check(ops, WORKLOADS[name], heads)
 
 
+@pytest.mark.parametrize("B,T,H", [
+    (1, 128, 12),    # one tile per head
+    (1, 129, 2),     # a 1-row tail
+    (2, 1000, 2),    # ragged, eight key tiles: seven ordered dq additions
+    (3, 640, 2),
+])
+def test_fused_backward_matches_oracle_and_split(ops, B, T, H):
+    """The fused backward (one pass; dq summed across CTAs in key-tile order)
+    against the oracle, and against the split backward: both compute the same
+    products and differ only in fp32 summation order."""
+    qkv_bf, dout_bf = make_inputs(B, T, H, 64, seed=31 + T)
+    qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
+    out, lse = ops.attn_fwd(qkv)
+    fused = torch.full_like(qkv, float("nan"))
+    ops.attn_bwd_fused(qkv, out, dout, lse, dqkv=fused)
+    split = ops.attn_bwd(qkv, out, dout, lse)
+    st, word = ops.last_device_status()
+    assert st == ops.GA_OK, (st, hex(word))
+    _, _, dqkv_o = orc.attention_forward_backward(qkv_bf.double().numpy(),
+                                                  dout_bf.double().numpy(), 0.125)
+    g_fused = fused.cpu().double().numpy()
+    g_split = split.cpu().double().numpy()
+    assert np.isfinite(g_fused).all()
+    for s_ in range(3):
+        assert rel_fro(g_fused[:, :, s_], dqkv_o[:, :, s_]) <= GRAD_TOL
+        assert rel_fro(g_fused[:, :, s_], g_split[:, :, s_]) <= 5e-3
+
+
+def test_fused_backward_full_size_and_deterministic(ops):
+    """At the bench shape (1536 items over a persistent grid: every query tile
+    gets up to eight ordered additions from CTAs in different rounds), sampled
+    heads against the oracle, and two runs bitwise equal."""
+    wl = WORKLOADS["gpt2-124m-b16-t1024"]
+    qkv_bf, dout_bf = make_inputs(wl.B, wl.T, wl.H, wl.D, seed=0)
+    qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
+    out, lse = ops.attn_fwd(qkv)
+    ws = torch.empty(ops.bwd_fused_workspace_size(wl.B, wl.T, wl.H, wl.D), dtype=torch.uint8,
+                     device="cuda")
+    a = ops.attn_bwd_fused(qkv, out, dout, lse, workspace=ws)
+    b = ops.attn_bwd_fused(qkv, out, dout, lse, workspace=ws)
+    st, word = ops.last_device_status()
+    assert st == ops.GA_OK, (st, hex(word))
+    assert torch.equal(a, b)
+    q64, d64 = qkv_bf.double().numpy(), dout_bf.double().numpy()
+    g = a.cpu().double().numpy()
+    for bb, hh in [(0, 0), (15, 11)]:
+        Q, K, V = (q64[bb, :, s_, hh] for s_ in range(3))
+        dQ, dK, dV = orc.head_backward(Q, K, V, d64[bb, :, hh], wl.scale)
+        for s_, ref in enumerate((dQ, dK, dV)):
+            assert rel_fro(g[bb, :, s_, hh], ref) <= GRAD_TOL
+
+
 def test_backward_is_deterministic(ops):
     qkv_bf, dout_bf = make_inputs(2, 1024, 3, 64, seed=11)
     qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
