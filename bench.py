@@ -22,6 +22,11 @@ collective.
 
 --impl reference times the CPU oracle (fp64 NumPy) on a bounded sample of the
 same workload on this host's cores.
+
+--decode times decode attention instead (gpt2_attn_decode: the newest row
+t = T-1 of every (b, h) over the keys and values of rows 0..T-1), one GPU,
+and prints its own line: bytes of k and v read per second against the
+measured HBM copy bandwidth.
 """
 
 from __future__ import annotations
@@ -468,6 +473,62 @@ def run_e2e(args, wl, ops, dev, qkv_cpu, dout_cpu, step_flops, world):
             "ms_per_step": ms / K}
 
 
+def run_decode(args, wl):
+    import torch
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from causal_self_attention_flashattention_b200 import build
+    build.build()
+    from causal_self_attention_flashattention_b200 import ops
+    from causal_self_attention_flashattention_b200.workload import make_inputs
+
+    B, T, H, D, scale = wl.B, wl.T, wl.H, wl.D, wl.scale
+    t = T - 1
+    qkv_cpu, _ = make_inputs(B, T, H, D, seed=0, qk_std=wl.qk_std)
+    # Rotating qkv buffers: 4 x 75 MB > L2, so each step reads k and v from HBM.
+    sets = [qkv_cpu.to(dev) for _ in range(args.sets)]
+    out = torch.empty(B, H, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, H, dtype=torch.float32, device=dev)
+    ws = torch.empty(ops.decode_workspace_size(B, T, H, D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        ops.attn_decode(sets[i % len(sets)], t, scale, out=out, lse=lse, workspace=ws, stream=stream)
+    torch.cuda.synchronize()
+    st, word = ops.last_device_status()
+    if st != ops.GA_OK:
+        raise RuntimeError(f"device status after warm-up: {ops.status_string(st)} ({word:#x})")
+    K = args.steps
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for i in range(K):
+        ops.attn_decode(sets[i % len(sets)], t, scale, out=out, lse=lse, workspace=ws, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / K
+    kv_bytes = 2 * B * H * (t + 1) * D * 2          # k and v rows 0..t, bf16
+    step_bytes = kv_bytes + B * H * D * 2 * 2 + B * H * 4  # + q read, out write, lse write
+    peaks, peak_src = load_peaks()
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "decode attention: bytes of q, k, v read and out, lse written per second",
+        "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "B": B, "T": T, "H": H, "D": D, "t": t,
+                   "l2": f"{len(sets)} rotating qkv buffers of {qkv_cpu.numel() * 2} B > 126 MB L2",
+                   "step": "gpt2_attn_decode (partial per 256-key chunk, then combine)"},
+        "roofline": {"kernel": "decode", "bound": "hbm", "achieved": gbs,
+                     "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                     "frac": gbs / float(peaks["hbm_gbs"]), "peak_source": f"hbm_gbs of {peak_src}",
+                     "algorithmic_bytes": step_bytes},
+        "gpu_launches": 2 * K,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
@@ -481,6 +542,8 @@ def main(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
+    p.add_argument("--decode", action="store_true",
+                   help="time decode attention (gpt2_attn_decode) instead")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be at least 3")
@@ -489,6 +552,8 @@ def main(argv=None):
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.decode:
+        return run_decode(args, wl)
     return run_ours(args, wl)
 
 

@@ -21,6 +21,7 @@
 #include "fwd.cuh"
 #include "bwd.cuh"
 #include "bwd_fused.cuh"
+#include "decode.cuh"
 
 namespace {
 
@@ -305,6 +306,39 @@ ga_status gpt2_attn_bwd(const void* qkv, const void* out, const void* dout, cons
   if ((st = gpt2_attn_bwd_dkdv(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream)) != GA_OK)
     return st;
   return gpt2_attn_bwd_dq(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
+}
+
+ga_status gpt2_attn_decode_workspace_size(int B, int T, int H, int D, size_t* bytes) {
+  if (bytes == nullptr) return GA_ERR_INVALID_ARG;
+  const ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  *bytes = ga::decode::ws_bytes(B, T, H);
+  return GA_OK;
+}
+
+ga_status gpt2_attn_decode(const void* qkv, int t, void* out, float* lse, void* workspace,
+                           size_t workspace_bytes, int B, int T, int H, int D, float scale,
+                           gpt2attn_stream_t stream) {
+  if (qkv == nullptr || out == nullptr || lse == nullptr) return GA_ERR_INVALID_ARG;
+  ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if ((st = check_scale(scale)) != GA_OK) return st;
+  if (t < 0 || t >= T || B > 65535 || H > 65535) return GA_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < ga::decode::ws_bytes(B, T, H))
+    return GA_ERR_WORKSPACE;
+  if (!aligned16(qkv) || !aligned16(out) || !aligned16(lse) || !aligned16(workspace))
+    return GA_ERR_ALIGNMENT;
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GA_ERR_CUDA;
+  const ga::AttnShape sh = make_shape(B, T, H, scale);
+  const int n_chunks = ga::decode::num_chunks(t);
+  float* partials = static_cast<float*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ga::decode::attn_decode_partial_kernel<<<dim3(n_chunks, H, B), ga::decode::kWarps * 32, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(qkv), t, partials, sh);
+  ga::decode::attn_decode_combine_kernel<<<dim3(H, B), ga::kD, 0, s>>>(
+      partials, n_chunks, static_cast<__nv_bfloat16*>(out), lse, sh);
+  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
 }
 
 ga_status gpt2_attn_last_device_status(gpt2attn_stream_t stream, unsigned long long* detail) {

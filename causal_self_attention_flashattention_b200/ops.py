@@ -44,6 +44,8 @@ EXPORTED_SYMBOLS = (
     "gpt2_attn_bwd_preprocess",
     "gpt2_attn_bwd_dkdv",
     "gpt2_attn_bwd_dq",
+    "gpt2_attn_decode_workspace_size",
+    "gpt2_attn_decode",
     "gpt2_attn_last_device_status",
     "gpt2_attn_status_string",
     "gpt2_attn_version",
@@ -76,6 +78,10 @@ _lib.gpt2_attn_bwd_dq.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _
 _lib.gpt2_attn_bwd_dq.restype = _i
 _lib.gpt2_attn_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
 _lib.gpt2_attn_bwd_noalloc.restype = _i
+_lib.gpt2_attn_decode_workspace_size.argtypes = [_i, _i, _i, _i, ctypes.POINTER(ctypes.c_size_t)]
+_lib.gpt2_attn_decode_workspace_size.restype = _i
+_lib.gpt2_attn_decode.argtypes = [_vp, _i, _vp, _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_decode.restype = _i
 _lib.gpt2_attn_last_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
 _lib.gpt2_attn_last_device_status.restype = _i
 _lib.gpt2_attn_status_string.argtypes = [_i]
@@ -314,6 +320,39 @@ def attn_bwd_noalloc(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
                                       lse.data_ptr(), dqkv.data_ptr(), B, T, H, D, scale,
                                       _stream_ptr(stream)), "gpt2_attn_bwd_noalloc")
     return dqkv
+
+
+def decode_workspace_size(B: int, T: int, H: int, D: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.gpt2_attn_decode_workspace_size(B, T, H, D, ctypes.byref(n)),
+           "gpt2_attn_decode_workspace_size")
+    return int(n.value)
+
+
+def attn_decode(qkv: torch.Tensor, t: int, scale: float | None = None,
+                out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None):
+    """Decode attention of query row ``t`` over rows 0..t of ``qkv``.
+
+    Returns (out (B,H,D) bf16, lse (B,H) fp32): row t of ``attn_fwd``'s result.
+    """
+    B, T, H, D = _dims(qkv)
+    _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
+    scale = default_scale(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.bfloat16, device=qkv.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=qkv.device)
+    _expect(out, "out", (B, H, D), torch.bfloat16)
+    _expect(lse, "lse", (B, H), torch.float32)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_size(B, T, H, D), dtype=torch.uint8,
+                                device=qkv.device)
+    ws, ws_bytes = _workspace(workspace)
+    _check(_lib.gpt2_attn_decode(qkv.data_ptr(), int(t), out.data_ptr(), lse.data_ptr(), ws,
+                                 ws_bytes, B, T, H, D, scale, _stream_ptr(stream)),
+           "gpt2_attn_decode")
+    return out, lse
 
 
 def last_device_status(stream=None) -> tuple[int, int]:

@@ -167,6 +167,28 @@ ga_status gpt2_attn_bwd_fused(const void* qkv, const void* dout, const float* ls
                               gpt2attn_stream_t stream);
 
 /*
+ * Decode attention: the attention output of query row t alone, over the keys
+ * and values of rows 0..t of the same packed qkv buffer (the newest token of a
+ * generation step, with the earlier rows' k and v kept in the buffer). This is
+ * row t of gpt2_attn_fwd's result, computed without the other rows.
+ *   qkv   [in]  bf16 (B,T,3,H,D), device; rows 0..t are read (q only of row t)
+ *   t     [in]  0 <= t < T
+ *   out   [out] bf16 (B,H,D), device
+ *   lse   [out] fp32 (B,H), device: natural log of sum_j exp(scale q.k_j)
+ *   workspace [scratch] >= gpt2_attn_decode_workspace_size bytes, 16-byte
+ *         aligned, not shared by calls that run concurrently
+ * Two launches on `stream`: per 256-key chunk of each (b,h), partial max, sum
+ * and unnormalised output (fp32, CUDA cores: the step is bound by reading k
+ * and v); then one combine per (b,h). GA_ERR_INVALID_ARG for t outside
+ * [0, T) or B, H above 65535.
+ */
+ga_status gpt2_attn_decode_workspace_size(int B, int T, int H, int D, size_t* bytes);
+ga_status gpt2_attn_decode(const void* qkv, int t, void* out, float* lse,
+                           void* workspace, size_t workspace_bytes,
+                           int B, int T, int H, int D, float scale,
+                           gpt2attn_stream_t stream);
+
+/*
  * gpt2_attn_bwd without a workspace argument, for callers that cannot
  * allocate device memory: a plugin that is handed only its input and output
  * buffers by a host application that owns all device memory, or a program

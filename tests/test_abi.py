@@ -115,3 +115,21 @@ def test_workspace_size():
     assert ops.lib().gpt2_attn_bwd_workspace_size(1, 8, 1, 48, ctypes.byref(n)) == ops.GA_ERR_UNSUPPORTED
     with pytest.raises(ops.AttnError):
         ops.bwd_workspace_size(0, 8, 1, 64)
+
+
+def test_decode_arguments_rejected_before_launch():
+    lib = ops.lib()
+    p = 1 << 20  # a 16-byte-aligned fake address: nothing is launched on these paths
+    n = ctypes.c_size_t(0)
+    assert lib.gpt2_attn_decode_workspace_size(2, 1000, 3, 64, ctypes.byref(n)) == ops.GA_OK
+    # partials fp32 [B][H][ceil(T/256)][2 + D]
+    assert n.value == 2 * 3 * 4 * 66 * 4
+    ws = n.value
+    assert lib.gpt2_attn_decode(p, 1000, p, p, p, ws, 2, 1000, 3, 64, 0.125, None) == ops.GA_ERR_INVALID_ARG
+    assert lib.gpt2_attn_decode(p, -1, p, p, p, ws, 2, 1000, 3, 64, 0.125, None) == ops.GA_ERR_INVALID_ARG
+    assert lib.gpt2_attn_decode(p, 5, p, p, p, ws - 4, 2, 1000, 3, 64, 0.125, None) == ops.GA_ERR_WORKSPACE
+    assert lib.gpt2_attn_decode(p, 5, p, p, None, ws, 2, 1000, 3, 64, 0.125, None) == ops.GA_ERR_WORKSPACE
+    assert lib.gpt2_attn_decode(p, 5, p, p + 4, p, ws, 2, 1000, 3, 64, 0.125, None) == ops.GA_ERR_ALIGNMENT
+    assert lib.gpt2_attn_decode(p, 5, p, p, p, ws, 2, 1000, 3, 32, 0.125, None) == ops.GA_ERR_UNSUPPORTED
+    assert lib.gpt2_attn_decode(None, 5, p, p, p, ws, 2, 1000, 3, 64, 0.125, None) == ops.GA_ERR_INVALID_ARG
+    assert lib.gpt2_attn_decode(p, 5, p, p, p, ws, 2, 1000, 3, 64, 0.0, None) == ops.GA_ERR_INVALID_ARG

@@ -204,6 +204,43 @@ def test_fused_backward_full_size_and_deterministic(ops):
             assert rel_fro(g[bb, :, s_, hh], ref) <= GRAD_TOL
 
 
+@pytest.mark.parametrize("B,T,H,ts", [
+    (1, 1, 1, [0]),                      # a single token
+    (2, 300, 3, [0, 1, 127, 255, 256, 299]),   # chunk edges (256 keys) and the last row
+    (1, 1000, 2, [511, 512, 999]),
+])
+def test_decode_matches_oracle_row(ops, B, T, H, ts):
+    """Decode attention of row t equals row t of the causal forward: out and
+    lse against the oracle, at chunk boundaries and the last row."""
+    qkv_bf, _ = make_inputs(B, T, H, 64, seed=40 + T)
+    qkv = qkv_bf.cuda()
+    out_o, lse_o = orc.attention_forward(qkv_bf.double().numpy(), 0.125)
+    ws = torch.empty(ops.decode_workspace_size(B, T, H, 64), dtype=torch.uint8, device="cuda")
+    for t in ts:
+        out, lse = ops.attn_decode(qkv, t, workspace=ws)
+        st, word = ops.last_device_status()
+        assert st == ops.GA_OK, (st, hex(word))
+        ok, err, _ = out_error_ok(out.cpu().double().numpy(), out_o[:, t])
+        assert ok, (t, err)
+        assert np.max(np.abs(lse.cpu().double().numpy() - lse_o[:, :, t])) <= LSE_TOL
+
+
+def test_decode_full_size_rows(ops):
+    """The bench shape: sampled rows against the oracle, head by head."""
+    wl = WORKLOADS["gpt2-124m-b16-t1024"]
+    qkv_bf, _ = make_inputs(wl.B, wl.T, wl.H, wl.D, seed=1)
+    qkv = qkv_bf.cuda()
+    q64 = qkv_bf.double().numpy()
+    for t in (1023, 640):
+        out, lse = ops.attn_decode(qkv, t)
+        for b, h in [(0, 0), (9, 7), (15, 11)]:
+            Q, K, V = (q64[b, :, s_, h] for s_ in range(3))
+            O, L, _ = orc.head_forward(Q, K, V, wl.scale)
+            assert out_error_ok(out[b, h].cpu().double().numpy(), O[t])[0]
+            assert abs(float(lse[b, h]) - L[t]) <= LSE_TOL
+    assert ops.last_device_status() == (ops.GA_OK, 0)
+
+
 def test_backward_is_deterministic(ops):
     qkv_bf, dout_bf = make_inputs(2, 1024, 3, 64, seed=11)
     qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
