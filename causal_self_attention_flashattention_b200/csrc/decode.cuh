@@ -13,12 +13,13 @@
 // more than 1/128 full). Keys are split into 256-row chunks (split-K):
 //   attn_decode_partial_kernel  one CTA (4 warps) per (chunk, h, b). The
 //       chunk's v rows are copied to shared memory (cp.async, 16 bytes per
-//       copy) while each warp scores its 64 keys (one key per lane, the q row
-//       in shared memory), so both loads are in flight at once. Each warp
-//       takes its max and sum in base 2 and accumulates p * v from shared
-//       memory, each lane owning two of the 64 columns; the four warps are then
-//       combined, and the chunk's (max, sum, unnormalised o) goes to the
-//       workspace.
+//       copy) while each warp scores its 64 keys, so both loads are in flight
+//       at once. Eight lanes read one 128-byte k row together (each 16 bytes
+//       against its eighth of q, then three shuffles), so a warp's load
+//       instruction covers four whole rows. Each warp takes its max and sum in
+//       base 2 and accumulates p * v from shared memory, each lane owning two
+//       of the 64 columns; the four warps are then combined, and the chunk's
+//       (max, sum, unnormalised o) goes to the workspace.
 //   attn_decode_combine_kernel  one CTA per (h, b): merges the chunks
 //       (rescaling each by 2^(m_c - m)) into out (bf16) and the natural-log lse.
 #pragma once
@@ -51,25 +52,6 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Score of one key row: q . k in fp32 (q as 32 bf16 pairs in registers).
-__device__ __forceinline__ float dot_row(const uint32_t (&q)[kD / 2],
-                                         const __nv_bfloat16* __restrict__ krow) {
-  const uint4* k4 = reinterpret_cast<const uint4*>(krow);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int c = 0; c < kD / 8; ++c) {
-    const uint4 w = __ldg(k4 + c);
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t qq = q[4 * c + e];
-      acc[e] = fmaf(__uint_as_float(qq << 16), __uint_as_float(u[e] << 16), acc[e]);
-      acc[e] = fmaf(__uint_as_float(qq & 0xFFFF0000u), __uint_as_float(u[e] & 0xFFFF0000u), acc[e]);
-    }
-  }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
-}
-
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
                : "memory");
@@ -79,6 +61,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 attn_decode_partial_kernel(const __nv_bfloat16* __restrict__ qkv, int t,
                            float* __restrict__ partials, const AttnShape sh) {
   __shared__ float m_s[kWarps], l_s[kWarps];
+  __shared__ float s_s[kWarps][64];  // the warps' scores
   __shared__ float o_s[kWarps][kD];
   __shared__ __align__(16) __nv_bfloat16 v_s[kChunk][kD];  // 32 KiB
   const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -96,25 +79,35 @@ attn_decode_partial_kernel(const __nv_bfloat16* __restrict__ qkv, int t,
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
-  uint32_t q[kD / 2];
-  {
-    const uint4* q4 = reinterpret_cast<const uint4*>(base + t * row_elems);
-#pragma unroll
-    for (int c = 0; c < kD / 8; ++c) {
-      const uint4 w = __ldg(q4 + c);
-      q[4 * c] = w.x;
-      q[4 * c + 1] = w.y;
-      q[4 * c + 2] = w.z;
-      q[4 * c + 3] = w.w;
-    }
-  }
+  // This lane's eighth of q: columns [8 * piece, 8 * piece + 8).
+  const int piece = lane & 7;
+  const uint4 qw = __ldg(reinterpret_cast<const uint4*>(base + t * row_elems) + piece);
+  const uint32_t q[4] = {qw.x, qw.y, qw.z, qw.w};
 
-  // Scores of this warp's 64 keys, two per lane (key0 = lane, key1 = lane + 32).
+  // Scores of this warp's 64 keys, four rows per step: lanes 8r..8r+7 read
+  // row r of the step, 16 bytes each.
   const int k0 = chunk * kChunk + warp * 64;
-  const int ka = k0 + lane, kb = k0 + 32 + lane;
   const __nv_bfloat16* kbase = base + sh.H * kD;  // the k slot
-  const float sa = ka <= t ? dot_row(q, kbase + ka * row_elems) * sh.scale_log2 : -INFINITY;
-  const float sb = kb <= t ? dot_row(q, kbase + kb * row_elems) * sh.scale_log2 : -INFINITY;
+#pragma unroll 4
+  for (int g = 0; g < 16; ++g) {
+    const int key = k0 + 4 * g + (lane >> 3);
+    float part = 0.f;
+    if (key <= t) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(kbase + key * row_elems) + piece);
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        part = fmaf(__uint_as_float(q[e] << 16), __uint_as_float(u[e] << 16), part);
+        part = fmaf(__uint_as_float(q[e] & 0xFFFF0000u), __uint_as_float(u[e] & 0xFFFF0000u), part);
+      }
+    }
+    part += __shfl_xor_sync(0xffffffffu, part, 4);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    if (piece == 0) s_s[warp][4 * g + (lane >> 3)] = key <= t ? part * sh.scale_log2 : -INFINITY;
+  }
+  __syncwarp();
+  const float sa = s_s[warp][lane], sb = s_s[warp][32 + lane];
   const float m = warp_max(fmaxf(sa, sb));
   // A warp whose keys all lie past t contributes nothing (m = -inf).
   const float pa = m == -INFINITY ? 0.f : exp2f(sa - m);
