@@ -310,7 +310,7 @@ def run_ours(args, wl):
         raise RuntimeError(f"device status after warm-up: {ops.status_string(st)} ({word:#x})")
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     sampler = None
@@ -326,7 +326,7 @@ def run_ours(args, wl):
     t_start.record(stream)
     for i in range(K):
         step(sets[i % n_sets], evs[i])
-    evs[-1][4].record(stream)
+    evs[-1][3].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
@@ -338,7 +338,7 @@ def run_ours(args, wl):
         raise RuntimeError(f"device status after timing: {ops.status_string(st)} ({word:#x})")
 
     total_ms = t_start.elapsed_time(t_end)
-    names = ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"]
+    names = ["fwd", "bwd_dq", "bwd_dkdv"]
     per = {n: 0.0 for n in names}
     for ev in evs:
         for k, n in enumerate(names):
@@ -366,9 +366,10 @@ def run_ours(args, wl):
     qkv_bytes = 3 * o_bytes
     kbytes = {
         "fwd": fwd_bytes,
-        "bwd_preprocess": 2 * o_bytes + lse_bytes,
+        # q, k, v, dO read; dk, dv written; lse and Delta read.
         "bwd_dkdv": qkv_bytes + o_bytes + 2 * lse_bytes + 2 * o_bytes,
-        "bwd_dq": qkv_bytes + o_bytes + 2 * lse_bytes + o_bytes,
+        # q, k, v, dO, O and lse read; dq and Delta written.
+        "bwd_dq": qkv_bytes + 2 * o_bytes + 2 * lse_bytes + o_bytes,
     }
     kernels = {}
     for n in names:
@@ -410,8 +411,8 @@ def run_ours(args, wl):
                              f"({n_sets * (2 * qkv_bytes + 3 * o_bytes) / 1e9:.2f} GB; "
                              f"{2 * qkv_bytes + 3 * o_bytes + 2 * lse_bytes} B touched per step) "
                              "> 126 MB L2",
-                       "step": "gpt2_attn_fwd + gpt2_attn_bwd (preprocess, dK/dV, dQ)"},
-            "clocks": clocks, "e2e": e2e, "gpu_launches": 4 * K,
+                       "step": "gpt2_attn_fwd + gpt2_attn_bwd (dQ with Delta, dK/dV)"},
+            "clocks": clocks, "e2e": e2e, "gpu_launches": 3 * K,
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu,
             "wall_s_timed_region": wall,
         }

@@ -8,14 +8,17 @@
 // where Delta_i = sum_j P_ij dP_ij = dO_i . O_i (the row term of the softmax
 // Jacobian, computed from out and dout).
 //
-// Three kernels, launched in this order on one stream:
-//   attn_bwd_pre_kernel  Delta[b,h,t] = sum_d dO o O, fp32 (memory bound).
+// Two kernels, launched in this order on one stream:
+//   attn_bwd_dq_kernel   one CTA per 128-query tile i: computes the tile's
+//                        Delta from its dO and O tiles (and writes it out),
+//                        streams key tiles j <= i, accumulates dQ in tensor
+//                        memory.
 //   attn_bwd_dkdv_kernel one CTA per 128-key tile j: streams query tiles
-//                        i >= j, accumulates dK and dV in tensor memory.
-//   attn_bwd_dq_kernel   one CTA per 128-query tile i: streams key tiles
-//                        j <= i, accumulates dQ in tensor memory. Nothing is
-//                        accumulated through atomics, so the result is
-//                        bitwise deterministic.
+//                        i >= j (reading Delta), accumulates dK and dV in
+//                        tensor memory.
+// Nothing is accumulated through atomics, so the result is bitwise
+// deterministic. attn_bwd_pre_kernel computes Delta on its own, for callers
+// of the separate preprocessing step and for the fused backward.
 #pragma once
 
 #include "common.cuh"
@@ -590,6 +593,7 @@ namespace dq {
 struct alignas(1024) Smem {
   uint8_t q[2][kTileBytes];  // [item slot]
   uint8_t dout[2][kTileBytes];
+  uint8_t o[2][kTileBytes];  // the forward's output tile, for Delta
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   uint64_t in_full[2], in_empty[2];
@@ -597,10 +601,49 @@ struct alignas(1024) Smem {
   uint64_t sdp_full, sdp_free, ds_full, acc_done;
   uint64_t ds_free[2];  // dS buffer b no longer read by a dQ product
   uint64_t drain[2];
+  uint64_t dpart_full[2];  // [item slot] the four Delta partial sums are in place
   uint32_t tmem_base;
   int abort;
 };
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+static_assert(kSmemBytes <= 232448, "dQ shared memory exceeds the 227 KiB per-block limit");
+
+// Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile.
+__device__ __forceinline__ int sw128_chunk(int r, int c) {
+  return (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4);
+}
+
+// Column group g's share of Delta for query row r: sum over columns
+// [16g, 16g + 16) of dO[r][d] * O[r][d] (chunks 2g and 2g + 1 of each row).
+// Only this thread reads those O bytes, so it then leaves the partial sum in
+// the first word of its chunk 2g, where the other groups pick it up.
+__device__ __forceinline__ void delta_part(const uint8_t* dout_tile, uint8_t* o_tile, int r,
+                                           int g) {
+  const int off0 = sw128_chunk(r, 2 * g), off1 = sw128_chunk(r, 2 * g + 1);
+  const uint4 a0 = *reinterpret_cast<const uint4*>(dout_tile + off0);
+  const uint4 a1 = *reinterpret_cast<const uint4*>(dout_tile + off1);
+  const uint4 o0 = *reinterpret_cast<const uint4*>(o_tile + off0);
+  const uint4 o1 = *reinterpret_cast<const uint4*>(o_tile + off1);
+  const uint32_t ua[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+  const uint32_t uo[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    acc[e & 3] = fmaf(__uint_as_float(ua[e] << 16), __uint_as_float(uo[e] << 16), acc[e & 3]);
+    acc[e & 3] = fmaf(__uint_as_float(ua[e] & 0xFFFF0000u), __uint_as_float(uo[e] & 0xFFFF0000u),
+                      acc[e & 3]);
+  }
+  *reinterpret_cast<float*>(o_tile + off0) = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// Delta of row r: the four groups' partial sums, added in one fixed order.
+__device__ __forceinline__ float delta_sum(const uint8_t* o_tile, int r) {
+  const float p0 = *reinterpret_cast<const float*>(o_tile + sw128_chunk(r, 0));
+  const float p1 = *reinterpret_cast<const float*>(o_tile + sw128_chunk(r, 2));
+  const float p2 = *reinterpret_cast<const float*>(o_tile + sw128_chunk(r, 4));
+  const float p3 = *reinterpret_cast<const float*>(o_tile + sw128_chunk(r, 6));
+  return (p0 + p1) + (p2 + p3);
+}
 
 __device__ __forceinline__ void decode(int k, const AttnShape& sh, int n_qt, int& b, int& h,
                                        int& i) {
@@ -613,8 +656,9 @@ __device__ __forceinline__ void decode(int k, const AttnShape& sh, int n_qt, int
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
-                   const __grid_constant__ CUtensorMap map_do, const float* __restrict__ lse,
-                   const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv,
+                   const __grid_constant__ CUtensorMap map_do,
+                   const __grid_constant__ CUtensorMap map_o, const float* __restrict__ lse,
+                   float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv,
                    const AttnShape sh) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -642,6 +686,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
     for (int d = 0; d < 2; ++d) {
       mbar_init(&sm.ds_free[d], 1);
       mbar_init(&sm.drain[d], 1);
+      mbar_init(&sm.dpart_full[d], kEwWarps);
     }
     sm.abort = 0;
     fence_barrier_init();
@@ -650,6 +695,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&map_qkv);
     tma_prefetch_desc(&map_do);
+    tma_prefetch_desc(&map_o);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -671,9 +717,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
         decode(k, sh, n_qt, b, h, i);
         const int slot = it_cnt & 1;
         if (!mbar_wait(&sm.in_empty[slot], ((it_cnt >> 1) & 1) ^ 1, kSiteDqProducer, abort)) break;
-        mbar_arrive_expect_tx(&sm.in_full[slot], 2 * kTileBytes);
+        mbar_arrive_expect_tx(&sm.in_full[slot], 3 * kTileBytes);
         tma_load_3d(sm.q[slot], &map_qkv, &sm.in_full[slot], h * kD, i * kBlockM, b);
         tma_load_3d(sm.dout[slot], &map_do, &sm.in_full[slot], h * kD, i * kBlockM, b);
+        tma_load_3d(sm.o[slot], &map_o, &sm.in_full[slot], h * kD, i * kBlockM, b);
         ++it_cnt;
         for (int j = 0; j <= i; ++j, ++kv_it) {
           const int s = kv_it % kStages;
@@ -789,7 +836,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
     const uint32_t t_s = tmem + lb + 32 * g, t_dp = tmem + lb + 128 + 32 * g;
     const uint32_t t_ds0 = tmem + lb + 256 + 16 * g, t_dq = tmem + lb + 384 + 16 * g;
     const float sc = sh.scale_log2;
-    uint32_t sdp_cnt = 0, acc_cnt = 0, ds_cnt = 0;
+    uint32_t sdp_cnt = 0, acc_cnt = 0, ds_cnt = 0, it_cnt = 0;
     // The finished item whose dQ still sits in tensor memory: it is read out
     // while the next item's first tile is processed, just before that tile's
     // dS goes to tensor memory (after which the next dQ product overwrites
@@ -807,7 +854,29 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qkv,
       const size_t lrow = (static_cast<size_t>(b) * sh.H + h) * sh.T + row;
       // Rows past T get -lse = -inf (P = 0).
       const float nl = valid ? -lse[lrow] * kLog2e : -INFINITY;
-      const float nd = valid ? -delta[lrow] : 0.f;
+      // Delta of this row from the item's dO and O tiles (their in_full phase
+      // makes the TMA writes visible here): each column group sums a quarter
+      // of the columns, the partial sums meet in the O tile (which nothing
+      // else reads), and every group adds the four in the same order. The
+      // first group writes Delta out for the dK/dV kernel. The O slot is
+      // reloaded only after this item's last dQ product, long after these
+      // reads.
+      const int slot = it_cnt & 1;
+      const uint32_t item_parity = (it_cnt >> 1) & 1;
+      ok = mbar_wait(&sm.in_full[slot], item_parity, kSiteDqSoftmax, abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      delta_part(sm.dout[slot], sm.o[slot], r, g);
+      fence_proxy_async_smem();  // order these writes before the slot's next TMA load
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.dpart_full[slot]);
+      ok = mbar_wait(&sm.dpart_full[slot], item_parity, kSiteDqSoftmax, abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++it_cnt;
+      const float dl = delta_sum(sm.o[slot], r);
+      if (valid && g == 0) delta[lrow] = dl;
+      const float nd = valid ? -dl : 0.f;
       for (int j = 0; j <= i; ++j) {
         ok = mbar_wait(&sm.sdp_full, sdp_cnt & 1, kSiteDqSoftmax, abort);
         ok = __all_sync(0xffffffffu, ok);

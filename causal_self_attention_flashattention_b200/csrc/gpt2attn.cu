@@ -4,12 +4,13 @@
 //
 // Nothing here allocates device memory. The only process-wide state is a
 // per-device cache of the SM count and of the kernels' shared-memory opt-in,
-// guarded by a mutex, and the device status word the kernels write when a
-// bounded wait gives up.
+// guarded by a mutex, the device status word the kernels write when a bounded
+// wait gives up, and the code of the last failed CUDA call.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -37,13 +38,20 @@ struct DeviceInfo {
 std::mutex g_mutex;
 DeviceInfo g_devices[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+PFN_cuCtxGetCurrent_v4000 g_ctx_get_current = nullptr;
 
-// Per-device set-up, once: SM count and the dynamic shared-memory opt-in of
-// every kernel. Returns nullptr on failure.
-const DeviceInfo* device_info() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_mutex);
+// The last CUDA failure behind a GA_ERR_CUDA: the failing step in the high 32
+// bits (kCudaErr*), its cudaError_t or CUresult in the low 32 bits.
+std::atomic<unsigned long long> g_cuda_error{0};
+constexpr unsigned long long kCudaErrSetup = 1, kCudaErrTensorMap = 2, kCudaErrLaunch = 3;
+
+void record_cuda_error(unsigned long long step, unsigned int code) {
+  g_cuda_error.store((step << 32) | code, std::memory_order_relaxed);
+}
+
+// With g_mutex held: fills g_devices[dev] on its first use (SM count, the
+// dynamic shared-memory opt-in of every kernel). Returns nullptr on failure.
+const DeviceInfo* setup_device(int dev) {
   DeviceInfo& info = g_devices[dev];
   if (info.ready) return &info;
   if (g_encode == nullptr) {
@@ -54,6 +62,14 @@ const DeviceInfo* device_info() {
         q != cudaDriverEntryPointSuccess || fn == nullptr)
       return nullptr;
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if (g_ctx_get_current == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return nullptr;
+    g_ctx_get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
   }
   if (cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return nullptr;
@@ -84,6 +100,41 @@ const DeviceInfo* device_info() {
   return &info;
 }
 
+// The current device's set-up, done once. Returns nullptr on failure (the
+// failing CUDA call's code is recorded; 0 if a non-CUDA check failed).
+const DeviceInfo* device_info() {
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    record_cuda_error(kCudaErrSetup, static_cast<unsigned int>(e));
+    return nullptr;
+  }
+  const DeviceInfo* ready = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    ready = setup_device(dev);
+  }
+  if (ready == nullptr) {
+    const cudaError_t le = cudaGetLastError();
+    record_cuda_error(kCudaErrSetup, static_cast<unsigned int>(le));
+    return nullptr;
+  }
+  // Tensor-map encoding is a driver call and needs a current context. A host
+  // thread whose CUDA runtime calls so far needed none (a framework's worker
+  // thread, say) has none bound yet: bind the device's primary context, as
+  // the runtime itself would at its first launch. A context the caller made
+  // current is left alone.
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) {
+    const cudaError_t se = cudaSetDevice(dev);
+    if (se != cudaSuccess) {
+      record_cuda_error(kCudaErrSetup, static_cast<unsigned int>(se));
+      return nullptr;
+    }
+  }
+  return ready;
+}
+
 // 3-D bf16 tensor map {inner, T, B} with a {64, 128, 1} box, 128-byte swizzle
 // and zero fill outside the tensor (rows past T read as 0).
 bool make_map(CUtensorMap* map, const void* base, uint64_t inner, int T, int B) {
@@ -95,7 +146,16 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, int T, int B) 
                               dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) record_cuda_error(kCudaErrTensorMap, static_cast<unsigned int>(r));
   return r == CUDA_SUCCESS;
+}
+
+// After a launch: GA_OK, or GA_ERR_CUDA with the launch error recorded.
+ga_status check_launch() {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return GA_OK;
+  record_cuda_error(kCudaErrLaunch, static_cast<unsigned int>(e));
+  return GA_ERR_CUDA;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -153,7 +213,7 @@ ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse, int B, int T, in
   ga::fwd::attn_fwd_kernel<<<grid_for(items, info->num_sms), ga::fwd::kThreads,
                              ga::fwd::kSmemBytes, s>>>(
       map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh);
-  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+  return check_launch();
 }
 
 ga_status gpt2_attn_bwd_workspace_size(int B, int T, int H, int D, size_t* bytes) {
@@ -186,7 +246,7 @@ ga_status launch_pre(const void* out, const void* dout, float* delta, uint32_t* 
   ga::bwd::attn_bwd_pre_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta,
       counters, n_counters, sh);
-  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+  return check_launch();
 }
 
 }  // namespace
@@ -254,19 +314,23 @@ ga_status gpt2_attn_bwd_dkdv(const void* qkv, const void* dout, const float* lse
   ga::bwd::dkdv::attn_bwd_dkdv_kernel<<<L.grid, ga::bwd::kThreads, ga::bwd::dkdv::kSmemBytes,
                                         reinterpret_cast<cudaStream_t>(stream)>>>(
       L.map_qkv, L.map_do, lse, delta, static_cast<__nv_bfloat16*>(dqkv), L.sh);
-  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+  return check_launch();
 }
 
-ga_status gpt2_attn_bwd_dq(const void* qkv, const void* dout, const float* lse,
-                           const float* delta, void* dqkv, int B, int T, int H, int D,
-                           float scale, gpt2attn_stream_t stream) {
+ga_status gpt2_attn_bwd_dq(const void* qkv, const void* out, const void* dout,
+                           const float* lse, float* delta, void* dqkv, int B, int T, int H,
+                           int D, float scale, gpt2attn_stream_t stream) {
+  if (out == nullptr) return GA_ERR_INVALID_ARG;
+  if (!aligned16(out)) return GA_ERR_ALIGNMENT;
   BwdLaunch L;
   const ga_status st = prepare_bwd(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, &L);
   if (st != GA_OK) return st;
+  CUtensorMap map_o;
+  if (!make_map(&map_o, out, static_cast<uint64_t>(H) * kD, T, B)) return GA_ERR_CUDA;
   ga::bwd::dq::attn_bwd_dq_kernel<<<L.grid, ga::bwd::kThreads, ga::bwd::dq::kSmemBytes,
                                     reinterpret_cast<cudaStream_t>(stream)>>>(
-      L.map_qkv, L.map_do, lse, delta, static_cast<__nv_bfloat16*>(dqkv), L.sh);
-  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+      L.map_qkv, L.map_do, map_o, lse, delta, static_cast<__nv_bfloat16*>(dqkv), L.sh);
+  return check_launch();
 }
 
 ga_status gpt2_attn_bwd_fused(const void* qkv, const void* dout, const float* lse,
@@ -286,7 +350,7 @@ ga_status gpt2_attn_bwd_fused(const void* qkv, const void* dout, const float* ls
       reinterpret_cast<float*>(ws + ga::bwd::fused::ws_dq_offset(B, T, H)),
       reinterpret_cast<uint32_t*>(ws + ga::bwd::fused::ws_cnt_offset(B, T, H)),
       static_cast<__nv_bfloat16*>(dqkv), L.sh);
-  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+  return check_launch();
 }
 
 ga_status gpt2_attn_bwd(const void* qkv, const void* out, const void* dout, const float* lse,
@@ -302,10 +366,10 @@ ga_status gpt2_attn_bwd(const void* qkv, const void* out, const void* dout, cons
       !aligned16(dqkv) || !aligned16(workspace))
     return GA_ERR_ALIGNMENT;
   float* delta = static_cast<float*>(workspace);
-  if ((st = gpt2_attn_bwd_preprocess(out, dout, delta, B, T, H, D, stream)) != GA_OK) return st;
-  if ((st = gpt2_attn_bwd_dkdv(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream)) != GA_OK)
+  if ((st = gpt2_attn_bwd_dq(qkv, out, dout, lse, delta, dqkv, B, T, H, D, scale, stream)) !=
+      GA_OK)
     return st;
-  return gpt2_attn_bwd_dq(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
+  return gpt2_attn_bwd_dkdv(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
 }
 
 ga_status gpt2_attn_decode_workspace_size(int B, int T, int H, int D, size_t* bytes) {
@@ -338,7 +402,7 @@ ga_status gpt2_attn_decode(const void* qkv, int t, void* out, float* lse, void* 
       static_cast<const __nv_bfloat16*>(qkv), t, partials, sh);
   ga::decode::attn_decode_combine_kernel<<<dim3(H, B), ga::kD, 0, s>>>(
       partials, n_chunks, static_cast<__nv_bfloat16*>(out), lse, sh);
-  return cudaGetLastError() == cudaSuccess ? GA_OK : GA_ERR_CUDA;
+  return check_launch();
 }
 
 ga_status gpt2_attn_last_device_status(gpt2attn_stream_t stream, unsigned long long* detail) {
@@ -355,6 +419,10 @@ ga_status gpt2_attn_last_device_status(gpt2attn_stream_t stream, unsigned long l
   if (detail != nullptr) *detail = word;
   if (word == 0) return GA_OK;
   return (word >> 32) == ga::kFwdValueRange ? GA_ERR_RANGE : GA_ERR_TIMEOUT;
+}
+
+unsigned long long gpt2_attn_last_cuda_error(void) {
+  return g_cuda_error.exchange(0, std::memory_order_relaxed);
 }
 
 const char* gpt2_attn_status_string(ga_status s) {

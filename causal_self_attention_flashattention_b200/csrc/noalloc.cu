@@ -10,8 +10,8 @@
 //
 // The array is loaded with the library on every GPU that runs it and stays
 // resident until the process exits: kMaxDeltaElems floats (4 MiB) per device.
-// It is shared by every call. The preprocess step rewrites every Delta value a
-// call reads before the call reads it, so nothing has to be cleared between
+// It is shared by every call. The dQ step rewrites every Delta value a call
+// reads before the call reads it, so nothing has to be cleared between
 // calls, but two calls whose work overlaps on the GPU (different streams, or
 // different host threads on one device) race on the array.
 #include <cuda_runtime.h>
@@ -52,7 +52,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
-// Every argument is checked here, before the first of the three launches.
+// Every argument is checked here, before the first of the two launches.
 extern "C" ga_status gpt2_attn_bwd_noalloc(const void* qkv, const void* out, const void* dout,
                                            const float* lse, void* dqkv, int B, int T, int H,
                                            int D, float scale, gpt2attn_stream_t stream) {
@@ -69,9 +69,7 @@ extern "C" ga_status gpt2_attn_bwd_noalloc(const void* qkv, const void* out, con
     return GA_ERR_ALIGNMENT;
   float* delta = delta_scratch();
   if (delta == nullptr) return GA_ERR_CUDA;
-  ga_status st = gpt2_attn_bwd_preprocess(out, dout, delta, B, T, H, D, stream);
+  const ga_status st = gpt2_attn_bwd_dq(qkv, out, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
   if (st != GA_OK) return st;
-  st = gpt2_attn_bwd_dkdv(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
-  if (st != GA_OK) return st;
-  return gpt2_attn_bwd_dq(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
+  return gpt2_attn_bwd_dkdv(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
 }

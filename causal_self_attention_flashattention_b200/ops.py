@@ -42,6 +42,7 @@ EXPORTED_SYMBOLS = (
     "gpt2_attn_bwd_prepare",
     "gpt2_attn_bwd_fused",
     "gpt2_attn_bwd_preprocess",
+    "gpt2_attn_last_cuda_error",
     "gpt2_attn_bwd_dkdv",
     "gpt2_attn_bwd_dq",
     "gpt2_attn_decode_workspace_size",
@@ -70,11 +71,13 @@ _lib.gpt2_attn_bwd_prepare.restype = _i
 _lib.gpt2_attn_bwd_fused.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_size_t, _vp,
                                      _i, _i, _i, _i, _f, _vp]
 _lib.gpt2_attn_bwd_fused.restype = _i
+_lib.gpt2_attn_last_cuda_error.argtypes = []
+_lib.gpt2_attn_last_cuda_error.restype = ctypes.c_ulonglong
 _lib.gpt2_attn_bwd_preprocess.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp]
 _lib.gpt2_attn_bwd_preprocess.restype = _i
 _lib.gpt2_attn_bwd_dkdv.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
 _lib.gpt2_attn_bwd_dkdv.restype = _i
-_lib.gpt2_attn_bwd_dq.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_bwd_dq.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
 _lib.gpt2_attn_bwd_dq.restype = _i
 _lib.gpt2_attn_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
 _lib.gpt2_attn_bwd_noalloc.restype = _i
@@ -111,6 +114,10 @@ def version() -> int:
 
 
 def _check(status: int, where: str) -> None:
+    if status == GA_ERR_CUDA:
+        word = int(_lib.gpt2_attn_last_cuda_error())
+        step = {1: "device set-up", 2: "TMA descriptor", 3: "kernel launch"}.get(word >> 32, "?")
+        raise AttnError(status, f"{where} ({step}: CUDA code {word & 0xFFFFFFFF})")
     if status != GA_OK:
         raise AttnError(status, where)
 
@@ -260,12 +267,13 @@ def attn_bwd_fused(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor, lse
 def attn_bwd_split_steps(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
                          lse: torch.Tensor, delta: torch.Tensor, dqkv: torch.Tensor,
                          scale: float | None = None, stream=None, events=None) -> torch.Tensor:
-    """``attn_bwd`` as its three C-ABI steps (preprocess, dK/dV, dQ).
+    """``attn_bwd`` as its two C-ABI steps (dQ, which also writes Delta, then
+    dK/dV, which reads it).
 
     Same result as ``attn_bwd``. ``delta`` is a caller-owned fp32 (B,H,T)
-    tensor. If ``events`` (four CUDA events) is given, they are recorded on the
-    stream before, between and after the three launches, so each step can be
-    timed on the device.
+    tensor; on return it holds Delta. If ``events`` (three CUDA events) is
+    given, they are recorded on the stream before, between and after the two
+    launches, so each step can be timed on the device.
     """
     B, T, H, D = _dims(qkv)
     _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
@@ -280,8 +288,9 @@ def attn_bwd_split_steps(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tenso
     sp = _stream_ptr(stream)
     if events is not None:
         events[0].record(stream)
-    _check(_lib.gpt2_attn_bwd_preprocess(out.data_ptr(), dout.data_ptr(), delta.data_ptr(),
-                                         B, T, H, D, sp), "gpt2_attn_bwd_preprocess")
+    _check(_lib.gpt2_attn_bwd_dq(qkv.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                                 delta.data_ptr(), dqkv.data_ptr(), B, T, H, D, scale, sp),
+           "gpt2_attn_bwd_dq")
     if events is not None:
         events[1].record(stream)
     _check(_lib.gpt2_attn_bwd_dkdv(qkv.data_ptr(), dout.data_ptr(), lse.data_ptr(),
@@ -289,11 +298,6 @@ def attn_bwd_split_steps(qkv: torch.Tensor, out: torch.Tensor, dout: torch.Tenso
            "gpt2_attn_bwd_dkdv")
     if events is not None:
         events[2].record(stream)
-    _check(_lib.gpt2_attn_bwd_dq(qkv.data_ptr(), dout.data_ptr(), lse.data_ptr(),
-                                 delta.data_ptr(), dqkv.data_ptr(), B, T, H, D, scale, sp),
-           "gpt2_attn_bwd_dq")
-    if events is not None:
-        events[3].record(stream)
     return dqkv
 
 

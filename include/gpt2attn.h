@@ -97,9 +97,10 @@ ga_status gpt2_attn_bwd_workspace_size(int B, int T, int H, int D, size_t* bytes
  *   workspace [scratch] device, >= gpt2_attn_bwd_workspace_size bytes,
  *             16-byte aligned, owned by the caller, must not be shared by
  *             calls that run concurrently
- * Three launches on `stream` (the split backward below): Delta; dk and dv per
- * key tile, which recompute P from lse; dq per query tile, which recomputes P
- * and accumulates dq in tensor memory with no atomics. The result is bitwise
+ * Two launches on `stream` (the split backward below): dq per query tile,
+ * which also computes that tile's Delta, recomputes P from lse and
+ * accumulates dq in tensor memory with no atomics; then dk and dv per key
+ * tile, which read Delta and recompute P. The result is bitwise
  * deterministic.
  */
 ga_status gpt2_attn_bwd(const void* qkv, const void* out, const void* dout,
@@ -109,29 +110,34 @@ ga_status gpt2_attn_bwd(const void* qkv, const void* out, const void* dout,
                         gpt2attn_stream_t stream);
 
 /*
- * The three steps of gpt2_attn_bwd as separate calls, with the same argument
- * conventions. gpt2_attn_bwd is exactly these three, in this order, on one
- * stream. `delta` is fp32 (B,H,T), caller-owned, 16-byte aligned.
+ * The two steps of gpt2_attn_bwd as separate calls, with the same argument
+ * conventions. gpt2_attn_bwd is exactly gpt2_attn_bwd_dq followed by
+ * gpt2_attn_bwd_dkdv on one stream. `delta` is fp32 (B,H,T), caller-owned,
+ * 16-byte aligned, where delta[b,h,t] = sum_d dout[b,t,h,d] * out[b,t,h,d]
+ * (the row term sum_j P_ij dP_ij of the softmax Jacobian).
  *
- * gpt2_attn_bwd_preprocess: delta[b,h,t] = sum_d dout[b,t,h,d] * out[b,t,h,d]
- *   (the row term sum_j P_ij dP_ij of the softmax Jacobian).
+ * gpt2_attn_bwd_dq: writes dqkv slot 0 (dq) and delta [out]; dqkv slots 1
+ *   and 2 untouched. One CTA per 128-query tile computes the tile's delta
+ *   from its dout and out rows, recomputes P and dP for every key tile at or
+ *   before it and accumulates dq in tensor memory (no atomics).
  * gpt2_attn_bwd_dkdv: writes dqkv slots 1 (dk) and 2 (dv); slot 0 untouched.
- *   One CTA per 128-key tile recomputes P from lse for every query tile at or
- *   after it and accumulates dk, dv in tensor memory.
- * gpt2_attn_bwd_dq: writes dqkv slot 0 (dq); slots 1 and 2 untouched. One CTA
- *   per 128-query tile recomputes P and dP for every key tile at or before it
- *   and accumulates dq in tensor memory (no atomics).
+ *   Reads delta [in] (as written by gpt2_attn_bwd_dq or
+ *   gpt2_attn_bwd_preprocess). One CTA per 128-key tile recomputes P from
+ *   lse for every query tile at or after it and accumulates dk, dv in tensor
+ *   memory.
+ * gpt2_attn_bwd_preprocess: delta alone, in its own memory-bound launch
+ *   (for callers that need delta without dq).
  */
-ga_status gpt2_attn_bwd_preprocess(const void* out, const void* dout, float* delta,
-                                   int B, int T, int H, int D, gpt2attn_stream_t stream);
+ga_status gpt2_attn_bwd_dq(const void* qkv, const void* out, const void* dout,
+                           const float* lse, float* delta, void* dqkv,
+                           int B, int T, int H, int D, float scale,
+                           gpt2attn_stream_t stream);
 ga_status gpt2_attn_bwd_dkdv(const void* qkv, const void* dout, const float* lse,
                              const float* delta, void* dqkv,
                              int B, int T, int H, int D, float scale,
                              gpt2attn_stream_t stream);
-ga_status gpt2_attn_bwd_dq(const void* qkv, const void* dout, const float* lse,
-                           const float* delta, void* dqkv,
-                           int B, int T, int H, int D, float scale,
-                           gpt2attn_stream_t stream);
+ga_status gpt2_attn_bwd_preprocess(const void* out, const void* dout, float* delta,
+                                   int B, int T, int H, int D, gpt2attn_stream_t stream);
 
 /*
  * The fused backward: the same dqkv from one pass over the causal tiles
@@ -219,11 +225,21 @@ ga_status gpt2_attn_bwd_noalloc(const void* qkv, const void* out, const void* do
  * Returns GA_ERR_TIMEOUT if a kernel of this library gave up on a device-side
  * wait since the last call (the kernel then stopped early and its outputs are
  * undefined), GA_ERR_RANGE if the forward met a v entry outside the fp16
- * range, GA_ERR_CUDA if the synchronisation itself failed, GA_OK otherwise. If `detail` is non-null it receives the raw status word (0 when
- * clean; otherwise the high 32 bits name the kernel and wait site and the
- * low 32 bits the block index).
+ * range, GA_ERR_CUDA if the synchronisation itself failed, GA_OK otherwise.
+ * If `detail` is non-null it receives the raw status word (0 when clean;
+ * otherwise the high 32 bits name the kernel and wait site and the low 32
+ * bits the block index).
  */
 ga_status gpt2_attn_last_device_status(gpt2attn_stream_t stream, unsigned long long* detail);
+
+/*
+ * The CUDA failure behind the latest GA_ERR_CUDA returned by any entry point
+ * of this library (from any host thread), then cleared; 0 if none since the
+ * last read. High 32 bits: the failing step (1 device set-up, 2 TMA
+ * descriptor encoding, 3 kernel launch); low 32 bits: its cudaError_t (steps
+ * 1 and 3; 0 when a non-CUDA set-up check failed) or CUresult (step 2).
+ */
+unsigned long long gpt2_attn_last_cuda_error(void);
 
 /* Static, human-readable name of a status code. Never returns NULL. */
 const char* gpt2_attn_status_string(ga_status s);

@@ -94,6 +94,32 @@ def test_bwd_rejects(kw, status):
     assert bwd(**kw) == status
 
 
+def bwd_dq(qkv=P, out=P, dout=P, lse=P, delta=P, dqkv=P, B=1, T=128, H=12, D=64, scale=0.125):
+    return ops.lib().gpt2_attn_bwd_dq(qkv, out, dout, lse, delta, dqkv, B, T, H, D, scale, None)
+
+
+def bwd_dkdv(qkv=P, dout=P, lse=P, delta=P, dqkv=P, B=1, T=128, H=12, D=64, scale=0.125):
+    return ops.lib().gpt2_attn_bwd_dkdv(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(out=None), ops.GA_ERR_INVALID_ARG),
+    (dict(delta=None), ops.GA_ERR_INVALID_ARG),
+    (dict(qkv=None), ops.GA_ERR_INVALID_ARG),
+    (dict(out=P_MIS), ops.GA_ERR_ALIGNMENT),
+    (dict(delta=P + 4), ops.GA_ERR_ALIGNMENT),
+    (dict(dqkv=P + 2), ops.GA_ERR_ALIGNMENT),
+    (dict(D=128), ops.GA_ERR_UNSUPPORTED),
+    (dict(T=0), ops.GA_ERR_INVALID_ARG),
+    (dict(scale=-0.5), ops.GA_ERR_INVALID_ARG),
+])
+def test_bwd_dq_rejects(kw, status):
+    # The dQ step reads out (for Delta) and writes delta; dK/dV reads delta.
+    assert bwd_dq(**kw) == status
+    if "out" not in kw:
+        assert bwd_dkdv(**kw) == status
+
+
 def _align256(x):
     return (x + 255) // 256 * 256
 

@@ -296,6 +296,28 @@ def test_delta_in_workspace(ops):
     assert np.allclose(delta_g, delta_o, rtol=1e-5, atol=1e-5)
 
 
+def test_split_steps_write_delta_for_dkdv(ops):
+    """gpt2_attn_bwd_dq writes every Delta the dK/dV step reads (a NaN-filled
+    delta buffer comes back finite), equal to the separate preprocess launch
+    up to fp32 summation order, and the two steps give attn_bwd's dqkv
+    bit for bit."""
+    B, T, H, D = 2, 333, 3, 64
+    qkv_bf, dout_bf = make_inputs(B, T, H, D, seed=9)
+    qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
+    out, lse = ops.attn_fwd(qkv)
+    delta = torch.full((B, H, T), float("nan"), dtype=torch.float32, device="cuda")
+    dqkv = torch.empty_like(qkv)
+    ops.attn_bwd_split_steps(qkv, out, dout, lse, delta, dqkv)
+    ref = torch.empty_like(delta)
+    assert ops.lib().gpt2_attn_bwd_preprocess(
+        out.data_ptr(), dout.data_ptr(), ref.data_ptr(), B, T, H, D, None) == ops.GA_OK
+    whole = ops.attn_bwd(qkv, out, dout, lse)
+    torch.cuda.synchronize()
+    assert torch.isfinite(delta).all()
+    assert torch.allclose(delta, ref, rtol=1e-6, atol=1e-6)
+    assert torch.equal(dqkv, whole)
+
+
 def test_runs_on_a_side_stream(ops):
     qkv_bf, dout_bf = make_inputs(1, 256, 2, 64, seed=6)
     s = torch.cuda.Stream()
@@ -305,6 +327,40 @@ def test_runs_on_a_side_stream(ops):
         dqkv = ops.attn_bwd(qkv, out, dout, lse)
     s.synchronize()
     out_o, lse_o, dqkv_o = orc.attention_forward_backward(
+        qkv_bf.double().numpy(), dout_bf.double().numpy(), 0.125)
+    assert out_error_ok(out.cpu().double().numpy(), out_o)[0]
+    assert rel_fro(dqkv.cpu().double().numpy(), dqkv_o) <= GRAD_TOL
+
+
+def test_calls_from_a_fresh_host_thread(ops):
+    """A host thread whose first CUDA work is this library's call has no
+    context bound yet (as in autograd's worker threads): the entry points bind
+    the device's primary context before encoding their tensor maps."""
+    import threading
+
+    B, T, H, D = 1, 200, 2, 64
+    qkv_bf, dout_bf = make_inputs(B, T, H, D, seed=8)
+    qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
+    out = torch.empty(B, T, H, D, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, H, T, dtype=torch.float32, device="cuda")
+    dqkv = torch.empty_like(qkv)
+    ws = torch.empty(ops.bwd_workspace_size(B, T, H, D), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    errors = []
+
+    def work():
+        try:
+            ops.attn_fwd(qkv, out=out, lse=lse, stream=stream)
+            ops.attn_bwd(qkv, out, dout, lse, dqkv=dqkv, workspace=ws, stream=stream)
+        except Exception as e:  # re-raised in the test's thread
+            errors.append(e)
+
+    t = threading.Thread(target=work)
+    t.start()
+    t.join()
+    assert not errors, errors
+    torch.cuda.synchronize()
+    out_o, _, dqkv_o = orc.attention_forward_backward(
         qkv_bf.double().numpy(), dout_bf.double().numpy(), 0.125)
     assert out_error_ok(out.cpu().double().numpy(), out_o)[0]
     assert rel_fro(dqkv.cpu().double().numpy(), dqkv_o) <= GRAD_TOL
