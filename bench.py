@@ -61,28 +61,39 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def csrc_digest() -> str:
-    csrc = os.path.join(ROOT, "causal_self_attention_flashattention_b200", "csrc")
+# The sources each kernel's code comes from: its own header plus the shared
+# helpers and the host file that configures its launch.
+KERNEL_SOURCES = {
+    "fwd": ("fwd.cuh",),
+    "bwd_dq": ("bwd.cuh",),
+    "bwd_dkdv": ("bwd.cuh",),
+    "bwd_prepare": ("bwd.cuh",),
+    "bwd_fused": ("bwd_fused.cuh", "bwd.cuh"),
+}
+COMMON_SOURCES = ("common.cuh", "ptx.cuh", "gpt2attn.cu")
+
+
+def kernel_digest(kernel: str, csrc: str | None = None) -> str:
+    """Digest of the sources a kernel is built from (changes when its code can)."""
+    csrc = csrc or os.path.join(ROOT, "causal_self_attention_flashattention_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in COMMON_SOURCES + KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
 def load_traffic():
-    """DRAM bytes per launch from the last committed ncu capture, or {} when the
-    kernel sources changed since that capture."""
+    """DRAM bytes per launch from the last committed ncu capture, for the
+    kernels whose sources are unchanged since that capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return {}
-    if d.get("csrc_digest") != csrc_digest():
-        return {}
-    return d.get("kernels", {})
+    return {k: v for k, v in d.get("kernels", {}).items()
+            if k in KERNEL_SOURCES and v.get("src_digest") == kernel_digest(k)}
 
 
 # ---------------------------------------------------------------------------

@@ -234,9 +234,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         if (n == 0) {
           // No second query tile in this item: this thread still releases its
           // share of the Q slot, after the slot's previous phase is complete
-          // (an earlier arrival could complete that phase instead).
+          // (an earlier arrival could complete that phase instead). It then
+          // waits for the other issuer to release the slot too, i.e. for the
+          // item to finish: every later wait of this thread is on a phase
+          // parity, which is only unambiguous while the barrier is at most one
+          // phase from the one expected. Skipping items without waiting let it
+          // run ahead of the Q and K/V loads of the next item it serves and
+          // read stale tiles.
           if (!mbar_wait(&sm.q_empty[slot], ((it_cnt >> 1) & 1) ^ 1, kSiteFwdMma, abort)) { ok = false; break; }
           mbar_arrive(&sm.q_empty[slot]);
+          if (!mbar_wait(&sm.q_empty[slot], (it_cnt >> 1) & 1, kSiteFwdMma, abort)) { ok = false; break; }
         } else {
           if (!mbar_wait(&sm.q_full[slot], (it_cnt >> 1) & 1, kSiteFwdMma, abort)) { ok = false; break; }
           tc_fence_after();

@@ -107,6 +107,19 @@ def test_fwd_bwd_matches_oracle(ops, B, T, H):
     check_all(ops, B, T, H, seed=B * 1000 + T)
 
 
+@pytest.mark.parametrize("B,T,H", [
+    (26, 384, 6),    # 312 items: pairs and lone last tiles on each CTA
+    (20, 640, 8),    # 480 items; CTAs 136-147 get two lone-tile items in a row
+    (40, 896, 4),    # 640 items, seven tiles
+])
+def test_several_items_per_cta(ops, B, T, H):
+    # More forward items (query-tile pairs) than CTAs with an odd tile count:
+    # the second query tile's issuer passes over items that have no second
+    # tile, and must not run ahead of the Q and K/V loads of the next item it
+    # serves (it once did and read stale tiles).
+    check_all(ops, B, T, H, seed=B + T + H)
+
+
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_small_gpt2_shape_seeds(ops, seed):
     check_all(ops, 1, 128, 12, seed=seed)
