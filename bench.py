@@ -3,8 +3,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME]
 
-One step = one forward (gpt2_attn_fwd) plus one backward (the three steps of
-gpt2_attn_bwd) over one batch of the GPT-2 124M training shape B=16, T=1024,
+One step = one forward (gpt2_attn_fwd) plus one backward (the two steps of
+gpt2_attn_bwd: dQ with Delta, then dK/dV) over one batch of the GPT-2 124M training shape B=16, T=1024,
 H=12, D=64, bf16 (seeded synthetic q, k, v, dO ~ N(0, 1)). The metric is
 causal attention fwd+bwd TFLOPS with the FLOPs counted as 2*B*H*T^2*D for the
 forward and 2.5x that for the backward, reported against the B200 dense bf16
@@ -14,7 +14,7 @@ Timing: W untimed warm-up steps, then exactly K steps between CUDA events on
 the launching stream, with a barrier and torch.cuda.synchronize() on both
 sides; the max over ranks is taken. Each step uses the next of four input/
 output buffer sets (~0.8 GB in all), so no step finds its inputs in the
-126 MB L2. Events recorded between the four launches of every step give each
+126 MB L2. Events recorded between the three launches of every step give each
 kernel's average duration, which feeds the roofline object. With --gpus N > 1
 (torchrun, one process per GPU) every rank runs its own replica: attention
 has no exchange step, so the scaling is weak and there is no data-path
@@ -266,6 +266,25 @@ def run_reference(args, wl):
 # ---------------------------------------------------------------------------
 # The CUDA path
 # ---------------------------------------------------------------------------
+def max_over_ranks(x: float, device) -> float:
+    """The maximum of x over all ranks of the process group (x itself when
+    there is none): a multi-rank time is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, steps: int, step_flops: float, ms: float) -> float:
+    """Whole-job throughput: every rank ran `steps` steps of `step_flops` in at
+    most `ms` milliseconds (weak scaling)."""
+    return world * steps * step_flops / (ms * 1e-3) / 1e12
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -356,14 +375,11 @@ def run_ours(args, wl):
             per[n] += ev[k].elapsed_time(ev[k + 1])
     per = {n: v / K for n, v in per.items()}
 
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
 
     fwd_flops, bwd_flops = attention_flops(B, T, H, D)
     step_flops = fwd_flops + bwd_flops
-    value = world * K * step_flops / (total_ms * 1e-3) / 1e12
+    value = job_tflops(world, K, step_flops, total_ms)
     peaks, peak_src = load_peaks()
     peak_tflops = float(peaks["bf16_tflops"])
 
@@ -508,13 +524,10 @@ def run_e2e(args, wl, ops, dev, qkv_cpu, dout_cpu, step_flops, world):
     st, word = ops.last_device_status()
     if st != ops.GA_OK:
         raise RuntimeError(f"device status after the end-to-end run: {ops.status_string(st)} ({word:#x})")
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     h2d = h_qkv.numel() * 2 + h_dout.numel() * 2
     d2h = sum(host_out[0][n].numel() * host_out[0][n].element_size() for n in ("out", "lse", "dqkv"))
-    return {"value": world * K * step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOPS",
+    return {"value": job_tflops(world, K, step_flops, ms), "unit": "TFLOPS",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
             "ms_per_step": ms / K,
             "pipeline": "2 device buffer sets; copy-in, compute and copy-out streams"}
