@@ -62,3 +62,70 @@ def test_exp2_poly_masked_and_underflow_inputs():
     y = np.array([-np.inf, -1e30, -300.0, -125.0, -124.9], dtype=np.float32)
     got = exp2_poly_model(y)
     assert np.all(np.isfinite(got)) and np.all(got > 0) and np.all(got < 2.0 ** -123)
+
+
+def _bf16_rne(x):
+    """float32 -> bf16 (as float32) with round to nearest even."""
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return (r & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
+
+
+def pack_f16_nonneg_model(p):
+    """float32/uint32 restatement of pack_f16_nonneg for one value: times
+    2^-112, add 0x1000 to the bits, keep bits [13, 29)."""
+    s = _const("kF32ToF16Scale")
+    m = (np.asarray(p, dtype=np.float32) * s).astype(np.float32)
+    b = (m.view(np.uint32).astype(np.uint64) + 0x1000) >> 13
+    assert np.all(b < 0x8000)   # no carry into the other half of the pair
+    return b.astype(np.uint16).view(np.float16)
+
+
+def test_f16_pack_scale_is_two_to_minus_112():
+    assert float(_const("kF32ToF16Scale")) == 2.0 ** -112
+
+
+def test_f16_pack_rounds_to_nearest_ties_away():
+    # Probabilities in [0, 2^8] (the stale-max bound). In fp16's normal range
+    # the 2^-112 multiply is exact, so the result is the correctly rounded
+    # value except that exact ties go up. Below 2^-14 the product is an fp32
+    # denormal, itself rounded to a 2^-37 grid (in p's units) first: the
+    # result is then within half an fp16 ulp plus 2^-37.
+    rng = np.random.default_rng(0)
+    p = np.concatenate([rng.uniform(0, 256, 200_000), rng.uniform(0, 2.0 ** -13, 50_000),
+                        np.array([0.0, 2.0 ** -24, 2.0 ** -14, 1.0, 255.875, 256.0])]).astype(np.float32)
+    got = pack_f16_nonneg_model(p).astype(np.float64)
+    exact = p.astype(np.float64)
+    ne = exact.astype(np.float16).astype(np.float64)          # round to nearest even
+    up = np.nextafter(ne.astype(np.float16), np.float16(np.inf)).astype(np.float64)
+    tie = np.abs(exact - ne) == np.abs(up - exact)
+    normal = exact >= 2.0 ** -14
+    assert np.all(got[normal & ~tie] == ne[normal & ~tie])
+    assert np.all(got[normal & tie] == np.maximum(ne[normal & tie], up[normal & tie]))
+    assert np.all(np.abs(got[~normal] - exact[~normal]) <= 2.0 ** -25 + 2.0 ** -37)
+    # Ties themselves: k + 1/2 fp16 ulps at 1.0 (ulp 2^-10) round up.
+    t = np.float32(1.0 + 2.0 ** -11)
+    assert float(pack_f16_nonneg_model(t)) == 1.0 + 2.0 ** -10
+
+
+def split3_bf16_model(v):
+    """float32 restatement of split3_bf16: three bf16 terms whose sum is v."""
+    v = np.asarray(v, dtype=np.float32)
+    h1 = _bf16_rne(v)
+    r1 = (v - h1).astype(np.float32)
+    h2 = _bf16_rne(r1)
+    h3 = _bf16_rne((r1 - h2).astype(np.float32))
+    return h1, h2, h3
+
+
+def test_split3_bf16_recovers_fp32_constants():
+    # The per-query constants folded into the dK/dV products (-lse*log2e-like
+    # values up to ~1e3 and -Delta): the three bf16 terms sum to v within
+    # 2^-24 of |v| in exact arithmetic, as the tensor core accumulates them.
+    rng = np.random.default_rng(1)
+    v = np.concatenate([rng.normal(0, 30, 100_000), rng.uniform(-1500, 1500, 100_000),
+                        rng.normal(0, 1e-3, 10_000)]).astype(np.float32)
+    h1, h2, h3 = split3_bf16_model(v)
+    total = h1.astype(np.float64) + h2.astype(np.float64) + h3.astype(np.float64)
+    err = np.abs(total - v.astype(np.float64))
+    assert np.all(err <= 2.0 ** -24 * np.abs(v.astype(np.float64)))
