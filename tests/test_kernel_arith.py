@@ -129,3 +129,27 @@ def test_split3_bf16_recovers_fp32_constants():
     total = h1.astype(np.float64) + h2.astype(np.float64) + h3.astype(np.float64)
     err = np.abs(total - v.astype(np.float64))
     assert np.all(err <= 2.0 ** -24 * np.abs(v.astype(np.float64)))
+
+
+def test_v_conversion_bf16_to_fp16_over_every_bf16_value():
+    # The forward rewrites V from bf16 to fp16 with a round-to-nearest-even
+    # conversion and flags a tile whose converted values include inf or NaN.
+    # Over all 65536 bf16 patterns: |v| <= 65504 converts exactly (fp16
+    # subnormals within 2^-25), and exactly the rest are flagged.
+    bits = np.arange(65536, dtype=np.uint32)
+    v = (bits << 16).astype(np.uint32).view(np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        h = v.astype(np.float16)
+    flagged = (h.view(np.uint16) & 0x7FFF) >= 0x7C00        # the kernel's inf/NaN test
+    fin = np.isfinite(v)
+    small = fin & (np.abs(v) <= 65504)
+    assert np.array_equal(flagged, ~small)
+    vv = v[small].astype(np.float64)
+    hh = h[small].astype(np.float64)
+    normal = np.abs(vv) >= 2.0 ** -14
+    assert np.all(hh[normal] == vv[normal])
+    assert np.all(np.abs(hh[~normal] - vv[~normal]) <= 2.0 ** -25)
+    # The boundary values of the GPU range test: 65280 passes, 65536 is flagged.
+    assert np.float16(np.float32(65280.0)) == 65280.0
+    with np.errstate(over="ignore"):
+        assert np.isinf(np.float16(np.float32(65536.0)))
