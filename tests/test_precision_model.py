@@ -100,3 +100,117 @@ def test_bf16_p_fails_the_stress_workload():
     okb, errb, _ = out_error_ok(kernel_forward_model(Q, K, V, 0.125, "bf16")[0].astype(np.float64), O)
     assert ok16 and not okb
     assert errb > 1.2e-2 > err16
+
+
+def _fma32(a, b, c):
+    """fp32 fused multiply-add: the exact a*b + c rounded once (two fp32
+    factors multiply exactly in fp64; the sum is rounded in fp64 first, which
+    differs from a single rounding only in rare ties)."""
+    return (np.asarray(a, np.float64) * np.asarray(b, np.float64) + np.asarray(c, np.float64)).astype(np.float32)
+
+
+def delta_model(dO, O):
+    """Delta of every row as the dQ kernel sums it: each 16-column group in
+    four fp32 accumulators (fused multiply-adds over the bf16 pairs), the
+    group's sum as (a0 + a1) + (a2 + a3), then the four groups the same way."""
+    dO = np.asarray(dO, np.float32)
+    O = np.asarray(O, np.float32)
+    parts = []
+    for g in range(4):
+        acc = [np.zeros(dO.shape[0], np.float32) for _ in range(4)]
+        for e in range(8):                        # 8 words = 16 columns
+            for half in (0, 1):
+                col = 16 * g + 2 * e + half
+                acc[e & 3] = _fma32(dO[:, col], O[:, col], acc[e & 3])
+        parts.append((acc[0] + acc[1]) + (acc[2] + acc[3]))
+    return (parts[0] + parts[1]) + (parts[2] + parts[3])
+
+
+def kernel_backward_model(Q, K, V, dO, out, lse, scale, fold_terms=3):
+    """fp32 restatement of the dQ and dK/dV kernels for one head (T a multiple
+    of 128), from the forward's bf16 out and fp32 lse. dK/dV folds -lse/scale
+    and -Delta into its products as `fold_terms` bf16 terms (3 in the kernel);
+    P and dS go to the tensor core as bf16."""
+    Q, K, V, dO, out = (np.asarray(a, np.float32) for a in (Q, K, V, dO, out))
+    lse = np.asarray(lse, np.float32)
+    T, D = Q.shape
+    nt = T // 128
+    sc = np.float32(np.float32(scale) * np.float32(LOG2E))
+    delta = delta_model(dO, out)
+    inv_scale = np.float32(1) / np.float32(scale)
+
+    def fold(v):
+        terms, r = [], v.astype(np.float32)
+        for _ in range(fold_terms):
+            t = _bf16_rne(r)
+            terms.append(t)
+            r = (r - t).astype(np.float32)
+        return np.sum(np.stack(terms).astype(np.float64), axis=0)
+
+    vl = fold((-lse * inv_scale).astype(np.float32))      # per query row
+    vd = fold(-delta)
+    nl = (-lse * np.float32(LOG2E)).astype(np.float32)
+    nd = -delta
+    dq = np.zeros((T, D), np.float32)
+    dk = np.zeros((T, D), np.float32)
+    dv = np.zeros((T, D), np.float32)
+    for i in range(nt):                 # query tile
+        qi, qs = slice(128 * i, 128 * i + 128), np.arange(128 * i, 128 * i + 128)
+        for j in range(i + 1):          # key tile
+            kj, ks = slice(128 * j, 128 * j + 128), np.arange(128 * j, 128 * j + 128)
+            S = (Q[qi] @ K[kj].T).astype(np.float32)
+            dP = (dO[qi] @ V[kj].T).astype(np.float32)
+            future = ks[None, :] > qs[:, None]
+            # dQ kernel: p = 2^(s*c - lse*log2e), dS = p * (dP - Delta)
+            with np.errstate(over="ignore"):
+                p_q = np.exp2(_fma32(S, sc, nl[qi, None]))
+            p_q[future] = 0
+            ds_q = _bf16_rne((p_q * (dP + nd[qi, None])).astype(np.float32))
+            dq[qi] = (dq[qi] + ds_q @ K[kj]).astype(np.float32)
+            # dK/dV kernel: the folded constants come out of the products
+            s_f = (S.astype(np.float64) + vl[qi, None]).astype(np.float32)
+            dp_f = (dP.astype(np.float64) + vd[qi, None]).astype(np.float32)
+            with np.errstate(over="ignore"):
+                p_k = np.exp2((s_f * sc).astype(np.float32))
+            p_k[future] = 0
+            pb = _bf16_rne(p_k)
+            db = _bf16_rne((p_k * dp_f).astype(np.float32))
+            dv[kj] = (dv[kj] + pb.T @ dO[qi]).astype(np.float32)
+            dk[kj] = (dk[kj] + db.T @ Q[qi]).astype(np.float32)
+    s = np.float32(scale)
+    return _bf16_rne(dq * s), _bf16_rne(dk * s), _bf16_rne(dv)
+
+
+def _rel_fro(g, o):
+    g = np.asarray(g, np.float64)
+    o = np.asarray(o, np.float64)
+    return np.linalg.norm(g - o) / np.linalg.norm(o)
+
+
+def _grads(B, T, H, qk_std, b, h, fold_terms=3):
+    qkv, dout = make_inputs(B, T, H, 64, seed=0, qk_std=qk_std)
+    q64, d64 = qkv.double().numpy(), dout.double().numpy()
+    Q, K, V = (q64[b, :, s, h] for s in range(3))
+    dO = d64[b, :, h]
+    out, lse = kernel_forward_model(Q, K, V, 0.125, "f16")
+    model = kernel_backward_model(Q, K, V, dO, out, lse, 0.125, fold_terms)
+    ref = orc.head_backward(Q, K, V, dO, 0.125)
+    return [_rel_fro(g, o) for g, o in zip(model, ref)]
+
+
+@pytest.mark.parametrize("B,T,H,qk_std,b,h", [
+    (16, 1024, 12, 1.0, 7, 5),      # the bench workload
+    (4, 4096, 12, 3.0, 3, 11),      # the stress workload
+])
+def test_backward_arithmetic_meets_the_gradient_tolerance(B, T, H, qk_std, b, h):
+    errs = _grads(B, T, H, qk_std, b, h)
+    assert max(errs) <= 2e-2, errs
+
+
+def test_one_term_fold_of_the_row_constants_would_not_do():
+    # Folding -lse/scale as a single bf16 term (its rounding error is up to
+    # 2^-9 of |lse|/scale, ~0.3 here) skews every P of the row; the three-term
+    # split keeps it to 2^-24.
+    three = _grads(4, 4096, 12, 3.0, 3, 11, fold_terms=3)
+    one = _grads(4, 4096, 12, 3.0, 3, 11, fold_terms=1)
+    assert max(one) > 2e-2 > max(three)
