@@ -23,10 +23,9 @@ collective.
 --impl reference times the CPU oracle (fp64 NumPy) on a bounded sample of the
 same workload on this host's cores.
 
---context times library attention on the same workload for comparison
-(flash-attn 2's packed-qkv function and torch's scaled_dot_product_attention,
-forward + backward through autograd) and prints one line per library. These
-are context figures, not this library's result.
+--context times torch's scaled_dot_product_attention (forward + backward
+through autograd) on the same workload and prints one line: a context
+figure, not this library's result.
 
 --decode times decode attention instead (gpt2_attn_decode: the newest row
 t = T-1 of every (b, h) over the keys and values of rows 0..T-1), one GPU,
@@ -595,7 +594,8 @@ def run_decode(args, wl):
 
 
 def run_context(args, wl):
-    """Library attention (fwd + bwd) on the same inputs, one JSON line each."""
+    """torch's scaled_dot_product_attention (fwd + bwd through autograd) on the
+    same inputs, as a context figure: one JSON line."""
     import torch
 
     from causal_self_attention_flashattention_b200.workload import attention_flops, make_inputs
@@ -607,39 +607,33 @@ def run_context(args, wl):
     sets = [(qkv_cpu.to(dev).requires_grad_(True), dout_cpu.to(dev)) for _ in range(args.sets)]
     fwd_flops, bwd_flops = attention_flops(B, T, H, D)
 
-    def fa2(qkv):
-        from flash_attn import flash_attn_qkvpacked_func
-        return flash_attn_qkvpacked_func(qkv, softmax_scale=scale, causal=True)
-
     def sdpa(qkv):
         q, k, v = (qkv[:, :, i].transpose(1, 2) for i in range(3))
         o = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True, scale=scale)
         return o.transpose(1, 2)
 
-    for name, fn in (("flash-attn 2 (qkvpacked)", fa2), ("torch SDPA", sdpa)):
-        line = {"impl": "context", "library": name, "metric": METRIC, "unit": "TFLOPS",
-                "config": {"workload": wl.name, "B": B, "T": T, "H": H, "D": D}}
-        try:
-            def step(i):
-                qkv, dout = sets[i % len(sets)]
-                out = fn(qkv)
-                torch.autograd.grad(out, qkv, dout)
-            for i in range(args.warmup):
-                step(i)
-            torch.cuda.synchronize()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            for i in range(args.steps):
-                step(i)
-            b.record()
-            torch.cuda.synchronize()
-            ms = a.elapsed_time(b) / args.steps
-            line.update(value=(fwd_flops + bwd_flops) / (ms * 1e-3) / 1e12, ms_per_step=ms,
-                        steps=args.steps)
-        except Exception as e:  # a library missing or without a kernel for this GPU
-            line["unavailable"] = f"{type(e).__name__}: {str(e).splitlines()[0][:160]}"
-        print(json.dumps(line), flush=True)
+    line = {"impl": "context", "library": "torch SDPA", "metric": METRIC, "unit": "TFLOPS",
+            "config": {"workload": wl.name, "B": B, "T": T, "H": H, "D": D}}
+    try:
+        def step(i):
+            qkv, dout = sets[i % len(sets)]
+            torch.autograd.grad(sdpa(qkv), qkv, dout)
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(args.steps):
+            step(i)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / args.steps
+        line.update(value=(fwd_flops + bwd_flops) / (ms * 1e-3) / 1e12, ms_per_step=ms,
+                    steps=args.steps)
+    except Exception as e:  # no kernel for this GPU in the installed torch
+        line["unavailable"] = f"{type(e).__name__}: {str(e).splitlines()[0][:160]}"
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -659,7 +653,7 @@ def main(argv=None):
     p.add_argument("--decode", action="store_true",
                    help="time decode attention (gpt2_attn_decode) instead")
     p.add_argument("--context", action="store_true",
-                   help="time library attention (flash-attn 2, torch SDPA) for comparison")
+                   help="time torch SDPA on the same workload, for context")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be at least 3")

@@ -35,6 +35,8 @@ enum WaitSite : uint32_t {
   kSiteFusedMma = 0x402,
   kSiteFusedSoftmax = 0x403,
   kSiteFusedDq = 0x404,  // waiting for earlier key tiles' dQ sums
+  kSiteSelftestWait = 0x501,  // the self-test's wait that nothing completes
+  kSiteSelftestPeer = 0x502,  // the self-test's second waiter (winds down on the abort flag)
 };
 
 struct AttnShape {

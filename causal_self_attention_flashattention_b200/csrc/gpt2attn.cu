@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "gpt2attn.h"
+#include "checks.h"
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -23,6 +24,26 @@
 #include "bwd.cuh"
 #include "bwd_fused.cuh"
 #include "decode.cuh"
+#include "selftest.cuh"
+
+namespace ga_host {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ga_status check_shape(int B, int T, int H, int D) {
+  if (B < 1 || T < 1 || H < 1 || D < 1) return GA_ERR_INVALID_ARG;
+  if (D != ga::kD) return GA_ERR_UNSUPPORTED;
+  const long double elems = static_cast<long double>(B) * T * 3 * H * D;
+  if (elems >= 2147483648.0L) return GA_ERR_INVALID_ARG;
+  return GA_OK;
+}
+
+ga_status check_scale(float scale) {
+  if (!std::isfinite(scale) || !(scale > 0.f)) return GA_ERR_INVALID_ARG;
+  return GA_OK;
+}
+
+}  // namespace ga_host
 
 namespace {
 
@@ -158,21 +179,9 @@ ga_status check_launch() {
   return GA_ERR_CUDA;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// Shape and scale checks shared by every entry point.
-ga_status check_shape(int B, int T, int H, int D) {
-  if (B < 1 || T < 1 || H < 1 || D < 1) return GA_ERR_INVALID_ARG;
-  if (D != kD) return GA_ERR_UNSUPPORTED;
-  const long double elems = static_cast<long double>(B) * T * 3 * H * D;
-  if (elems >= 2147483648.0L) return GA_ERR_INVALID_ARG;
-  return GA_OK;
-}
-
-ga_status check_scale(float scale) {
-  if (!std::isfinite(scale) || !(scale > 0.f)) return GA_ERR_INVALID_ARG;
-  return GA_OK;
-}
+using ga_host::aligned16;
+using ga_host::check_scale;
+using ga_host::check_shape;
 
 ga::AttnShape make_shape(int B, int T, int H, float scale) {
   ga::AttnShape sh;
@@ -402,6 +411,14 @@ ga_status gpt2_attn_decode(const void* qkv, int t, void* out, float* lse, void* 
       static_cast<const __nv_bfloat16*>(qkv), t, partials, sh);
   ga::decode::attn_decode_combine_kernel<<<dim3(H, B), ga::kD, 0, s>>>(
       partials, n_chunks, static_cast<__nv_bfloat16*>(out), lse, sh);
+  return check_launch();
+}
+
+ga_status gpt2_attn_selftest_wait_timeout(unsigned long long limit_ns, gpt2attn_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > ga::kMaxSelftestLimitNs) return GA_ERR_INVALID_ARG;
+  if (device_info() == nullptr) return GA_ERR_CUDA;
+  ga::selftest::wait_timeout_kernel<<<1, ga::selftest::kThreads, 0,
+                                      reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
   return check_launch();
 }
 

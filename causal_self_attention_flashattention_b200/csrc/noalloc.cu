@@ -16,11 +16,11 @@
 // different host threads on one device) race on the array.
 #include <cuda_runtime.h>
 
-#include <cmath>
 #include <cstdint>
 #include <mutex>
 
 #include "gpt2attn.h"
+#include "checks.h"
 
 namespace {
 
@@ -48,28 +48,28 @@ float* delta_scratch() {
   return g_delta_ptr[dev];
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 
-// Every argument is checked here, before the first of the two launches.
+// Every argument is checked here, with the same rules as every other entry
+// point (checks.h), before the first of the two launches; only the size limit
+// of the static array is this entry point's own.
 extern "C" ga_status gpt2_attn_bwd_noalloc(const void* qkv, const void* out, const void* dout,
                                            const float* lse, void* dqkv, int B, int T, int H,
                                            int D, float scale, gpt2attn_stream_t stream) {
-  if (B < 1 || T < 1 || H < 1 || D < 1) return GA_ERR_INVALID_ARG;
-  if (D != 64) return GA_ERR_UNSUPPORTED;
-  if (static_cast<long double>(B) * T * 3 * H * D >= 2147483648.0L) return GA_ERR_INVALID_ARG;
+  ga_status st = ga_host::check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
   if (static_cast<long double>(B) * H * T > static_cast<long double>(kMaxDeltaElems))
     return GA_ERR_WORKSPACE;
   if (qkv == nullptr || out == nullptr || dout == nullptr || lse == nullptr || dqkv == nullptr)
     return GA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || scale == INFINITY) return GA_ERR_INVALID_ARG;
-  if (!aligned16(qkv) || !aligned16(out) || !aligned16(dout) || !aligned16(lse) ||
-      !aligned16(dqkv))
+  if ((st = ga_host::check_scale(scale)) != GA_OK) return st;
+  if (!ga_host::aligned16(qkv) || !ga_host::aligned16(out) || !ga_host::aligned16(dout) ||
+      !ga_host::aligned16(lse) || !ga_host::aligned16(dqkv))
     return GA_ERR_ALIGNMENT;
   float* delta = delta_scratch();
   if (delta == nullptr) return GA_ERR_CUDA;
-  const ga_status st = gpt2_attn_bwd_dq(qkv, out, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
-  if (st != GA_OK) return st;
+  if ((st = gpt2_attn_bwd_dq(qkv, out, dout, lse, delta, dqkv, B, T, H, D, scale, stream)) !=
+      GA_OK)
+    return st;
   return gpt2_attn_bwd_dkdv(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, stream);
 }

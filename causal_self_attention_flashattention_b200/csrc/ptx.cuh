@@ -105,11 +105,12 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete. Returns false (after
-// recording `site`) on timeout, or when another role of the CTA has already
-// raised `*abort`.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t site,
-                                          volatile int* abort) {
+// Waits for the phase with the given parity to complete, for at most
+// `limit_ns`. Returns false (after recording `site` and raising `*abort`) when
+// the limit passes, or (without recording) when another role of the CTA has
+// already raised `*abort`.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, uint32_t site,
+                                                volatile int* abort, uint64_t limit_ns) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -117,13 +118,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     if (mbar_try_wait_sleep(addr, parity, kWaitSleepNs)) return true;
     if ((it & 7u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitTimeoutNs) {
+      if (globaltimer() - t0 > limit_ns) {
         record_failure(site);
         *abort = 1;
         return false;
       }
     }
   }
+}
+
+// The wait every kernel of the library uses: mbar_wait_limit with the 2 s
+// limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t site,
+                                          volatile int* abort) {
+  return mbar_wait_limit(bar, parity, site, abort, kWaitTimeoutNs);
 }
 
 // Wait used while winding down: ignores the abort flag, still bounded.
@@ -470,6 +478,40 @@ __device__ __forceinline__ uint32_t max_abs_f16x2(uint32_t a, uint32_t b) {
 
 // Magnitude bits of an fp16 at or above this: inf or NaN.
 constexpr uint32_t kF16InfBits = 0x7C00u;
+
+// Per 16-bit half: the larger of a and b as unsigned integers.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// bf16 magnitude bits (per half) at or above this: |v| > 65280, the largest
+// bf16 that fp16 holds (the next bf16, 65536, is beyond fp16's 65504), or inf,
+// or NaN.
+constexpr uint32_t kBf16BeyondF16 = 0x4780u;
+
+// A pair of bf16 values (low half first) to a pair of fp16 values with
+// integer operations only, leaving the exp unit to the softmax. A bf16 with
+// biased exponent e and mantissa m is 2^(e-127) (1 + m/128); its fp16 has
+// exponent e - 112 and mantissa m << 3, i.e. fp16 magnitude bits =
+// (bf16 magnitude bits - (112 << 7)) << 3. Both halves go through one 32-bit
+// multiply-add: (mag - 0x38003800) * 8 == mag * 8 + 0x3FFE4000 (mod 2^32),
+// with no carry or borrow between the halves while each half's magnitude lies
+// in [0x3800, 0x477F]; magnitudes below are clamped up to 0x3800, and above
+// it the range tracker is raised (the pair's value is then unspecified).
+// Results:
+//   2^-14 <= |v| <= 65280   exact (every such bf16 is an fp16 normal);
+//   |v| < 2^-15             +-0 (the clamp maps it to 0x3800, i.e. fp16 0);
+//   2^-15 <= |v| < 2^-14    an fp16 subnormal within 2^-15 of v;
+//   |v| > 65280, inf, NaN   unspecified, and `rng` (a running per-half max of
+//                           the magnitude bits) reaches kBf16BeyondF16.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u, uint32_t& rng) {
+  const uint32_t mag = u & 0x7FFF7FFFu;
+  rng = max_u16x2(rng, mag);
+  const uint32_t clamped = max_u16x2(mag, 0x38003800u);
+  return (clamped * 8u + 0x3FFE4000u) | (u & 0x80008000u);
+}
 
 // Warpgroup-wide register budget changes (all four warps of a warpgroup
 // execute the same one). The budgets of all warpgroups must add up to no more

@@ -48,6 +48,7 @@ EXPORTED_SYMBOLS = (
     "gpt2_attn_decode_workspace_size",
     "gpt2_attn_decode",
     "gpt2_attn_last_device_status",
+    "gpt2_attn_selftest_wait_timeout",
     "gpt2_attn_status_string",
     "gpt2_attn_version",
 )
@@ -87,6 +88,8 @@ _lib.gpt2_attn_decode.argtypes = [_vp, _i, _vp, _vp, _vp, ctypes.c_size_t, _i, _
 _lib.gpt2_attn_decode.restype = _i
 _lib.gpt2_attn_last_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
 _lib.gpt2_attn_last_device_status.restype = _i
+_lib.gpt2_attn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, _vp]
+_lib.gpt2_attn_selftest_wait_timeout.restype = _i
 _lib.gpt2_attn_status_string.argtypes = [_i]
 _lib.gpt2_attn_status_string.restype = ctypes.c_char_p
 _lib.gpt2_attn_version.argtypes = []

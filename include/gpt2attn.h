@@ -221,6 +221,24 @@ ga_status gpt2_attn_bwd_noalloc(const void* qkv, const void* out, const void* do
                                 gpt2attn_stream_t stream);
 
 /*
+ * Self-test of the device-side failure path that every kernel of this library
+ * shares. Launches one small kernel on `stream` in which one thread waits on
+ * a shared-memory barrier that nothing ever completes, bounded by
+ * `limit_ns` nanoseconds (0 < limit_ns <= 1e9, else GA_ERR_INVALID_ARG).
+ * When the limit passes, that thread records its wait site (0x501) in the
+ * device status word and raises the block's abort flag; a second waiter on
+ * the same barrier, bounded by the library's usual 2 s limit, sees the flag
+ * and returns without recording, and the block frees its tensor memory and
+ * exits. Nothing traps or faults, and the context stays usable.
+ * A following gpt2_attn_last_device_status returns GA_ERR_TIMEOUT with
+ * detail >> 32 == 0x501 (and clears the word). This is the same bounded wait
+ * the attention kernels use; this entry point exists so that the path that
+ * ends it can be exercised on purpose. It has no counterpart on the pages.
+ */
+ga_status gpt2_attn_selftest_wait_timeout(unsigned long long limit_ns,
+                                          gpt2attn_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word.
  * Returns GA_ERR_TIMEOUT if a kernel of this library gave up on a device-side
  * wait since the last call (the kernel then stopped early and its outputs are

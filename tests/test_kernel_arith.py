@@ -131,25 +131,72 @@ def test_split3_bf16_recovers_fp32_constants():
     assert np.all(err <= 2.0 ** -24 * np.abs(v.astype(np.float64)))
 
 
+def bf16x2_to_f16x2_model(u):
+    """uint32 restatement of bf16x2_to_f16x2 on packed pairs: magnitude mask,
+    per-half unsigned max with 0x3800 (clamp), one 32-bit multiply-add
+    (mag * 8 + 0x3FFE4000 mod 2^32), signs put back. Returns the packed fp16
+    pairs and the per-half magnitudes the range tracker sees."""
+    u = np.asarray(u, dtype=np.uint32)
+    mag = u & np.uint32(0x7FFF7FFF)
+    lo = np.maximum(mag & np.uint32(0xFFFF), np.uint32(0x3800))
+    hi = np.maximum(mag >> np.uint32(16), np.uint32(0x3800))
+    clamped = (hi << np.uint32(16)) | lo
+    z = (clamped.astype(np.uint64) * 8 + 0x3FFE4000) & 0xFFFFFFFF
+    r = z.astype(np.uint32) | (u & np.uint32(0x80008000))
+    return r, mag & np.uint32(0xFFFF), mag >> np.uint32(16)
+
+
+def _check_halves(v, h):
+    """Every in-range bf16 value v against the fp16 value h it became."""
+    v = v.astype(np.float64)
+    h = h.astype(np.float64)
+    normal = np.abs(v) >= 2.0 ** -14
+    assert np.all(h[normal] == v[normal])                     # exact
+    tiny = ~normal
+    assert np.all(np.abs(h[tiny] - v[tiny]) <= 2.0 ** -15)    # within 2^-15
+    assert np.all(h[np.abs(v) < 2.0 ** -15] == 0)             # flushed to +-0
+    assert np.all(np.signbit(h) == np.signbit(v))
+
+
 def test_v_conversion_bf16_to_fp16_over_every_bf16_value():
-    # The forward rewrites V from bf16 to fp16 with a round-to-nearest-even
-    # conversion and flags a tile whose converted values include inf or NaN.
-    # Over all 65536 bf16 patterns: |v| <= 65504 converts exactly (fp16
-    # subnormals within 2^-25), and exactly the rest are flagged.
+    # The forward rewrites V from bf16 to fp16 with integer operations only.
+    # Over all 65536 bf16 patterns, in the low and in the high half of a word
+    # (with an in-range partner in the other half): every |v| <= 65280 (the
+    # largest bf16 fp16 holds) converts exactly down to 2^-14 and within 2^-15
+    # below; the partner is unaffected; and exactly the patterns beyond that
+    # (|v| >= 65536, inf, NaN) raise the range tracker.
     bits = np.arange(65536, dtype=np.uint32)
-    v = (bits << 16).astype(np.uint32).view(np.float32)
-    with np.errstate(over="ignore", invalid="ignore"):
-        h = v.astype(np.float16)
-    flagged = (h.view(np.uint16) & 0x7FFF) >= 0x7C00        # the kernel's inf/NaN test
-    fin = np.isfinite(v)
-    small = fin & (np.abs(v) <= 65504)
-    assert np.array_equal(flagged, ~small)
-    vv = v[small].astype(np.float64)
-    hh = h[small].astype(np.float64)
-    normal = np.abs(vv) >= 2.0 ** -14
-    assert np.all(hh[normal] == vv[normal])
-    assert np.all(np.abs(hh[~normal] - vv[~normal]) <= 2.0 ** -25)
-    # The boundary values of the GPU range test: 65280 passes, 65536 is flagged.
-    assert np.float16(np.float32(65280.0)) == 65280.0
-    with np.errstate(over="ignore"):
-        assert np.isinf(np.float16(np.float32(65536.0)))
+    v = (bits << np.uint32(16)).view(np.float32)
+    in_range = np.isfinite(v) & (np.abs(v) <= 65280.0)
+    partner = np.uint32(0xBF40)                             # -0.75
+    for shift in (0, 16):
+        other = 16 - shift
+        words = (bits << np.uint32(shift)) | (partner << np.uint32(other))
+        r, mlo, mhi = bf16x2_to_f16x2_model(words)
+        m = mlo if shift == 0 else mhi
+        flagged = m >= 0x4780                                 # kBf16BeyondF16
+        assert np.array_equal(flagged, ~in_range)
+        h = ((r >> np.uint32(shift)) & np.uint32(0xFFFF)).astype(np.uint16).view(np.float16)
+        _check_halves(v[in_range], h[in_range])
+        p = ((r[in_range] >> np.uint32(other)) & np.uint32(0xFFFF)).astype(np.uint16).view(np.float16)
+        assert np.all(p.astype(np.float64) == -0.75)
+    # Boundary values: 65280 converts exactly, 65536 is flagged.
+    r, mlo, _ = bf16x2_to_f16x2_model(np.array([0x477F, 0x4780], dtype=np.uint32))
+    assert (r[0] & 0xFFFF).astype(np.uint16).view(np.float16) == 65280.0
+    assert mlo[0] < 0x4780 <= mlo[1]
+
+
+def test_v_conversion_random_pairs_both_halves():
+    # Random in-range pairs: both halves exact (or within 2^-15 when tiny).
+    rng = np.random.default_rng(3)
+    f = np.concatenate([rng.normal(0, 1, 200_000), rng.normal(0, 1e-4, 20_000),
+                        rng.uniform(-65280, 65280, 20_000)]).astype(np.float32)
+    b = (f.view(np.uint32) >> np.uint32(16)).astype(np.uint32)     # truncate to bf16
+    b = b[: (len(b) // 2) * 2].reshape(-1, 2)
+    words = b[:, 0] | (b[:, 1] << np.uint32(16))
+    r, mlo, mhi = bf16x2_to_f16x2_model(words)
+    assert np.all(mlo < 0x4780) and np.all(mhi < 0x4780)
+    for k, shift in enumerate((0, 16)):
+        v = (b[:, k] << np.uint32(16)).view(np.float32)
+        h = ((r >> np.uint32(shift)) & np.uint32(0xFFFF)).astype(np.uint16).view(np.float16)
+        _check_halves(v, h)

@@ -9,8 +9,7 @@ Tolerances (on bf16-rounded inputs that both sides see):
 Small shapes compare every element. Shapes that span several tiles and a
 ragged tail (T not a multiple of 128) cover the tail handling. The five GPT-2
 workload shapes run the full problem on the GPU, in the same launch
-configuration the benchmark times, and compare sampled heads with the oracle
-computed head by head.
+configuration the benchmark times, and compare every head with the oracle.
 """
 
 import numpy as np
@@ -134,35 +133,56 @@ def test_other_scale(ops):
     check_all(ops, 1, 300, 2, seed=9, scale=0.05)
 
 
-def sampled_heads_check(ops, wl, heads, seed=0):
+def host_cores():
+    import os
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def every_head_check(ops, wl, seed=0):
+    """The full workload on the GPU, in the launch configuration the bench
+    times, against the oracle on every (b, h): out and lse element by element,
+    dq/dk/dv relative Frobenius per head and per tensor."""
     qkv_bf, dout_bf = make_inputs(wl.B, wl.T, wl.H, wl.D, seed=seed, qk_std=wl.qk_std)
     out_g, lse_g, dqkv_g = run_gpu(ops, qkv_bf, dout_bf, wl.scale)
-    q64 = qkv_bf.double().numpy()
-    d64 = dout_bf.double().numpy()
-    for b, h in heads:
-        Q, K, V = (q64[b, :, s, h] for s in range(3))
-        O, lse, _ = orc.head_forward(Q, K, V, wl.scale)
-        dQ, dK, dV = orc.head_backward(Q, K, V, d64[b, :, h], wl.scale)
-        ok_out, err_out, n_floor = out_error_ok(out_g[b, :, h].double().numpy(), O)
-        assert ok_out, (b, h, err_out, n_floor)
-        assert np.max(np.abs(lse_g[b, h].double().numpy() - lse)) <= LSE_TOL
-        g = dqkv_g[b, :, :, h].double().numpy()
-        for s, ref in enumerate((dQ, dK, dV)):
-            assert rel_fro(g[:, s], ref) <= GRAD_TOL, (b, h, s, rel_fro(g[:, s], ref))
-    # Properties that hold at any size, over every head.
-    assert torch.isfinite(out_g.float()).all() and torch.isfinite(dqkv_g.float()).all()
-    # Query 0 attends only to key 0: out[:, 0] == v[:, 0] up to bf16 rounding.
-    assert torch.equal(out_g[:, 0], qkv_bf[:, 0, 2])
+    # The T x T matrices of one head at T = 4096 take ~1 GB of host memory in
+    # the oracle, so fewer workers run at once there.
+    procs = host_cores() if wl.T <= 1024 else min(host_cores(), 8)
+    out_o, lse_o, dqkv_o = orc.attention_forward_backward(
+        qkv_bf.double().numpy(), dout_bf.double().numpy(), wl.scale, processes=procs)
+    out_g = out_g.double().numpy()
+    ok_out, err_out, n_floor = out_error_ok(out_g, out_o)
+    assert ok_out, (err_out, n_floor)
+    err_lse = float(np.max(np.abs(lse_g.double().numpy() - lse_o)))
+    assert err_lse <= LSE_TOL, err_lse
+    worst = grads_every_head_ok(dqkv_g.double().numpy(), dqkv_o)
+    return err_out, err_lse, worst
 
 
-@pytest.mark.parametrize("name,heads", [
-    ("gpt2-124m-b16-t1024", [(0, 0), (7, 5), (15, 11)]),
-    ("gpt2-124m-b64-t1024", [(0, 3), (63, 11)]),
-    ("gpt2-350m-b32-t1024", [(1, 15), (31, 0)]),
-    ("stress-b4-t4096-qk3", [(0, 0), (3, 11)]),
+def grads_every_head_ok(g, dqkv_o):
+    """dq, dk, dv (B,T,3,H,D): relative Frobenius error <= GRAD_TOL for every
+    head of every slot, and for each slot over the whole batch."""
+    assert np.isfinite(g).all()
+    worst = []
+    for s in range(3):
+        diff = g[:, :, s] - dqkv_o[:, :, s]                  # (B, T, H, D)
+        num = np.sqrt(np.sum(diff * diff, axis=(1, 3)))      # per (b, h)
+        den = np.sqrt(np.sum(dqkv_o[:, :, s] ** 2, axis=(1, 3)))
+        per_head = num / np.where(den > 0, den, 1.0)
+        b, h = np.unravel_index(int(np.argmax(per_head)), per_head.shape)
+        worst.append(float(per_head[b, h]))
+        assert per_head.max() <= GRAD_TOL, ("slot", s, "head", (int(b), int(h)), worst[-1])
+        assert rel_fro(g[:, :, s], dqkv_o[:, :, s]) <= GRAD_TOL
+    return worst
+
+
+@pytest.mark.parametrize("name", [
+    "gpt2-124m-b16-t1024",     # the bench workload: 192 heads
+    "gpt2-124m-b64-t1024",     # 768 heads
+    "gpt2-350m-b32-t1024",     # 512 heads
+    "stress-b4-t4096-qk3",     # 48 heads of T = 4096, peaked rows
 ])
-def test_full_size_workloads_sampled_heads(ops, name, heads):
-    sampled_heads_check(ops, WORKLOADS[name], heads)
+def test_full_size_workloads_every_head(ops, name):
+    every_head_check(ops, WORKLOADS[name])
 
 
 @pytest.mark.parametrize("B,T,H", [
@@ -195,8 +215,8 @@ def test_fused_backward_matches_oracle_and_split(ops, B, T, H):
 
 def test_fused_backward_full_size_and_deterministic(ops):
     """At the bench shape (1536 items over a persistent grid: every query tile
-    gets up to eight ordered additions from CTAs in different rounds), sampled
-    heads against the oracle, and two runs bitwise equal."""
+    gets up to eight ordered additions from CTAs in different rounds), every
+    head against the oracle, and two runs bitwise equal."""
     wl = WORKLOADS["gpt2-124m-b16-t1024"]
     qkv_bf, dout_bf = make_inputs(wl.B, wl.T, wl.H, wl.D, seed=0)
     qkv, dout = qkv_bf.cuda(), dout_bf.cuda()
@@ -208,13 +228,9 @@ def test_fused_backward_full_size_and_deterministic(ops):
     st, word = ops.last_device_status()
     assert st == ops.GA_OK, (st, hex(word))
     assert torch.equal(a, b)
-    q64, d64 = qkv_bf.double().numpy(), dout_bf.double().numpy()
-    g = a.cpu().double().numpy()
-    for bb, hh in [(0, 0), (15, 11)]:
-        Q, K, V = (q64[bb, :, s_, hh] for s_ in range(3))
-        dQ, dK, dV = orc.head_backward(Q, K, V, d64[bb, :, hh], wl.scale)
-        for s_, ref in enumerate((dQ, dK, dV)):
-            assert rel_fro(g[bb, :, s_, hh], ref) <= GRAD_TOL
+    _, _, dqkv_o = orc.attention_forward_backward(
+        qkv_bf.double().numpy(), dout_bf.double().numpy(), wl.scale, processes=host_cores())
+    grads_every_head_ok(a.cpu().double().numpy(), dqkv_o)
 
 
 @pytest.mark.parametrize("B,T,H,ts", [
@@ -239,18 +255,17 @@ def test_decode_matches_oracle_row(ops, B, T, H, ts):
 
 
 def test_decode_full_size_rows(ops):
-    """The bench shape: sampled rows against the oracle, head by head."""
+    """The bench shape: rows t of every (b, h) against the oracle's forward."""
     wl = WORKLOADS["gpt2-124m-b16-t1024"]
     qkv_bf, _ = make_inputs(wl.B, wl.T, wl.H, wl.D, seed=1)
     qkv = qkv_bf.cuda()
-    q64 = qkv_bf.double().numpy()
-    for t in (1023, 640):
+    out_o, lse_o = orc.attention_forward(qkv_bf.double().numpy(), wl.scale,
+                                         processes=host_cores())
+    for t in (1023, 640, 255, 0):
         out, lse = ops.attn_decode(qkv, t)
-        for b, h in [(0, 0), (9, 7), (15, 11)]:
-            Q, K, V = (q64[b, :, s_, h] for s_ in range(3))
-            O, L, _ = orc.head_forward(Q, K, V, wl.scale)
-            assert out_error_ok(out[b, h].cpu().double().numpy(), O[t])[0]
-            assert abs(float(lse[b, h]) - L[t]) <= LSE_TOL
+        ok, err, _ = out_error_ok(out.cpu().double().numpy(), out_o[:, t])
+        assert ok, (t, err)
+        assert np.max(np.abs(lse.cpu().double().numpy() - lse_o[:, :, t])) <= LSE_TOL, t
     assert ops.last_device_status() == (ops.GA_OK, 0)
 
 
