@@ -27,6 +27,10 @@ same workload on this host's cores.
 through autograd) on the same workload and prints one line: a context
 figure, not this library's result.
 
+--fp8 times the FP8 forward (gpt2_attn_fwd_fp8) and its quantisation pass,
+with the bf16 forward on the same inputs for reference. --linear times the
+dense layers around attention (c_attn, c_proj) at the workload's B, T, C.
+
 --decode times decode attention instead (gpt2_attn_decode: the newest row
 t = T-1 of every (b, h) over the keys and values of rows 0..T-1), one GPU,
 and prints its own line: bytes of k and v read per second against the
@@ -372,6 +376,18 @@ def run_ours(args, wl):
         raise RuntimeError(f"device status after timing: {ops.status_string(st)} ({word:#x})")
 
     total_ms = t_start.elapsed_time(t_end)
+    # Host cost of issuing a step (the Python binding, the C-ABI argument
+    # checks, tensor-map lookups and three launches), without the per-kernel
+    # events: wall-clock time of K_h back-to-back steps before the device
+    # catches up, per step. At small shapes this, not the kernels, sets the
+    # step time.
+    k_host = min(K, 200)
+    torch.cuda.synchronize()
+    h0 = time.perf_counter()
+    for i in range(k_host):
+        step(sets[i % n_sets])
+    host_us = (time.perf_counter() - h0) / k_host * 1e6
+    torch.cuda.synchronize()
     names = ["fwd", "bwd_dq", "bwd_dkdv"]
     per = {n: 0.0 for n in names}
     for ev in evs:
@@ -444,6 +460,9 @@ def run_ours(args, wl):
                              "> 126 MB L2",
                        "step": "gpt2_attn_fwd + gpt2_attn_bwd (dQ with Delta, dK/dV)"},
             "clocks": clocks, "e2e": e2e, "gpu_launches": 3 * K,
+            "host": {"issue_us_per_step": host_us, "steps": k_host,
+                     "what": "wall-clock per step of issuing fwd + bwd from Python (binding, "
+                             "checks, tensor maps, 3 launches); not in the timed region"},
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu,
             "wall_s_timed_region": wall,
         }
@@ -593,6 +612,129 @@ def run_decode(args, wl):
     return 0
 
 
+def _time_device(fn, steps, warmup, stream):
+    """Average device time (ms) of fn() over `steps` calls on `stream`."""
+    import torch
+
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def run_fp8(args, wl):
+    """The FP8 forward (gpt2_attn_fwd_fp8) and its quantisation pass
+    (gpt2_attn_fp8_quantize), timed separately, next to the bf16 forward on the
+    same inputs: forward TFLOPS (2*B*H*T^2*D) against the dense e4m3 peak,
+    taken as the measured bf16 peak times 2, the nominal fp8/bf16 ratio."""
+    import torch
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from causal_self_attention_flashattention_b200 import build
+    build.build()
+    from causal_self_attention_flashattention_b200 import ops
+    from causal_self_attention_flashattention_b200.workload import attention_flops, make_inputs
+
+    B, T, H, D, scale = wl.B, wl.T, wl.H, wl.D, wl.scale
+    qkv_cpu, _ = make_inputs(B, T, H, D, seed=0, qk_std=wl.qk_std)
+    sets = []
+    for _ in range(args.sets):
+        qkv = qkv_cpu.to(dev)
+        qkv8, scales = ops.fp8_quantize(qkv)
+        sets.append(dict(qkv=qkv, qkv8=qkv8, scales=scales,
+                         out=torch.empty(B, T, H, D, dtype=torch.bfloat16, device=dev),
+                         lse=torch.empty(B, H, T, dtype=torch.float32, device=dev)))
+    stream = torch.cuda.current_stream()
+    n = len(sets)
+    ms_fp8 = _time_device(lambda i: ops.attn_fwd_fp8(sets[i % n]["qkv8"], sets[i % n]["scales"], scale,
+                                                     out=sets[i % n]["out"], lse=sets[i % n]["lse"],
+                                                     stream=stream), args.steps, args.warmup, stream)
+    ms_q = _time_device(lambda i: ops.fp8_quantize(sets[i % n]["qkv"], qkv8=sets[i % n]["qkv8"],
+                                                   scales=sets[i % n]["scales"], stream=stream),
+                        args.steps, args.warmup, stream)
+    ms_bf16 = _time_device(lambda i: ops.attn_fwd(sets[i % n]["qkv"], scale, out=sets[i % n]["out"],
+                                                  lse=sets[i % n]["lse"], stream=stream),
+                           args.steps, args.warmup, stream)
+    st, word = ops.last_device_status()
+    if st != ops.GA_OK:
+        raise RuntimeError(f"device status: {ops.status_string(st)} ({word:#x})")
+    fwd_flops, _ = attention_flops(B, T, H, D)
+    peaks, peak_src = load_peaks()
+    fp8_peak = 2.0 * float(peaks["bf16_tflops"])
+    tf = fwd_flops / (ms_fp8 * 1e-3) / 1e12
+    line = {
+        "metric": "causal attention FP8 forward TFLOPS (e4m3 q, k, v; per-tensor scales)",
+        "value": tf, "unit": "TFLOPS", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_fp8, "higher_is_better": True, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": wl.name, "B": B, "T": T, "H": H, "D": D,
+                   "l2": f"{n} rotating input sets"},
+        "roofline": {"kernel": "fwd_fp8", "bound": "tensor", "achieved": tf, "peak": fp8_peak,
+                     "unit": "TFLOP/s", "frac": tf / fp8_peak,
+                     "peak_source": f"bf16_tflops of {peak_src} x 2 (nominal e4m3/bf16 ratio)"},
+        "quantize_ms": ms_q, "bf16_fwd_ms": ms_bf16,
+        "gpu_launches": args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_linear(args, wl):
+    """The dense layers around attention (gpt2_attn_qkv_proj, gpt2_attn_out_proj)
+    at the workload's B, T and width C = 64 H: TFLOPS against the measured bf16
+    peak, one line each."""
+    import torch
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from causal_self_attention_flashattention_b200 import build
+    build.build()
+    from causal_self_attention_flashattention_b200 import ops
+    from causal_self_attention_flashattention_b200.workload import make_linear_inputs
+
+    B, T, H = wl.B, wl.T, wl.H
+    C = 64 * H
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    for name, n_out in (("c_attn (gpt2_attn_qkv_proj)", 3 * C), ("c_proj (gpt2_attn_out_proj)", C)):
+        x, w, b = make_linear_inputs(B, T, C, n_out, seed=0)
+        sets = [dict(x=x.to(dev), w=w.to(dev), b=b.to(dev),
+                     y=torch.empty(B, T, n_out, dtype=torch.bfloat16, device=dev))
+                for _ in range(args.sets)]
+        n = len(sets)
+        if n_out == 3 * C:
+            fn = lambda i: ops.qkv_proj(sets[i % n]["x"], sets[i % n]["w"], sets[i % n]["b"], H,
+                                        qkv=sets[i % n]["y"].view(B, T, 3, H, 64), stream=stream)
+        else:
+            fn = lambda i: ops.out_proj(sets[i % n]["x"].view(B, T, H, 64), sets[i % n]["w"],
+                                        sets[i % n]["b"], y=sets[i % n]["y"], stream=stream)
+        ms = _time_device(fn, args.steps, args.warmup, stream)
+        flops = 2.0 * B * T * C * n_out
+        tf = flops / (ms * 1e-3) / 1e12
+        print(json.dumps({
+            "metric": f"{name} TFLOPS", "value": tf, "unit": "TFLOPS", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "M": B * T, "N": n_out, "K": C,
+                       "l2": f"{n} rotating input/output sets"},
+            "roofline": {"kernel": "linear", "bound": "tensor", "achieved": tf, "peak": peak,
+                         "unit": "TFLOP/s", "frac": tf / peak,
+                         "peak_source": f"bf16_tflops (burst) of {peak_src}"},
+            "gpu_launches": args.steps}), flush=True)
+    st, word = ops.last_device_status()
+    if st != ops.GA_OK:
+        raise RuntimeError(f"device status: {ops.status_string(st)} ({word:#x})")
+    return 0
+
+
 def run_context(args, wl):
     """torch's scaled_dot_product_attention (fwd + bwd through autograd) on the
     same inputs, as a context figure: one JSON line."""
@@ -652,6 +794,10 @@ def main(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     p.add_argument("--decode", action="store_true",
                    help="time decode attention (gpt2_attn_decode) instead")
+    p.add_argument("--fp8", action="store_true",
+                   help="time the FP8 forward (and its quantisation pass) instead")
+    p.add_argument("--linear", action="store_true",
+                   help="time the dense layers around attention (c_attn, c_proj) instead")
     p.add_argument("--context", action="store_true",
                    help="time torch SDPA on the same workload, for context")
     args = p.parse_args(argv)
@@ -666,6 +812,10 @@ def main(argv=None):
         return run_decode(args, wl)
     if args.context:
         return run_context(args, wl)
+    if args.fp8:
+        return run_fp8(args, wl)
+    if args.linear:
+        return run_linear(args, wl)
     return run_ours(args, wl)
 
 

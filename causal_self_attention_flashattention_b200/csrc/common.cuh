@@ -35,6 +35,10 @@ enum WaitSite : uint32_t {
   kSiteFusedMma = 0x402,
   kSiteFusedSoftmax = 0x403,
   kSiteFusedDq = 0x404,  // waiting for earlier key tiles' dQ sums
+  kSiteDecode = 0x701,  // the decode kernel's wait for its k and v chunk
+  kSiteLinearProducer = 0x601,
+  kSiteLinearMma = 0x602,
+  kSiteLinearEpilogue = 0x603,
   kSiteSelftestWait = 0x501,  // the self-test's wait that nothing completes
   kSiteSelftestPeer = 0x502,  // the self-test's second waiter (winds down on the abort flag)
 };

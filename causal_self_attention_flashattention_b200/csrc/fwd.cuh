@@ -24,7 +24,8 @@
 //     grows, and writes P as fp16. No row statistic crosses a thread. At the
 //     end O is normalised and stored (bf16), and lse = ln2 * (m + log2 l).
 //   * Warp 11 (convert): rewrites each V tile in shared memory from bf16 to
-//     fp16 in place, so that O += P V runs as an fp16 x fp16 product. P in
+//     fp16 in place (or, in the FP8 forward, widens the e4m3 tile into a
+//     separate fp16 tile), so that O += P V runs as an fp16 x fp16 product. P in
 //     [0, 1] keeps 11 significant bits instead of 8, which matters on peaked
 //     rows where one probability near 1 multiplies a large v. Every bf16 value
 //     with |v| <= 65504 converts exactly (tiny ones to fp16 subnormals, within
@@ -70,10 +71,16 @@ __device__ __forceinline__ uint32_t col_s(int q) { return q * 128; }
 __device__ __forceinline__ uint32_t col_p(int q) { return 256 + q * 64; }
 __device__ __forceinline__ uint32_t col_o(int q) { return 384 + q * 64; }
 
+// Bytes of one 128 x 64 Q or K tile: bf16, or e4m3 in the FP8 forward.
+template <bool kFp8>
+constexpr int kQKBytes = kFp8 ? kTileBytes / 2 : kTileBytes;
+
+template <bool kFp8>
 struct alignas(1024) Smem {
-  uint8_t q[2][2][kTileBytes];   // [item slot][query tile]
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
+  uint8_t q[2][2][kQKBytes<kFp8>];   // [item slot][query tile]
+  uint8_t k[kStages][kQKBytes<kFp8>];
+  uint8_t v[kStages][kTileBytes];     // fp16 V as the P V product reads it
+  uint8_t v8[kStages][kFp8 ? kTileBytes / 2 : 16];  // e4m3 V as loaded (FP8 only)
   uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[kStages], kv_empty[kStages], v_ready[kStages];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
@@ -82,7 +89,8 @@ struct alignas(1024) Smem {
   int abort;
 };
 
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
+template <bool kFp8>
+constexpr size_t kSmemBytes = sizeof(Smem<kFp8>) + 1024;  // + alignment slack
 
 struct Item {
   int b, h, i0, has1, n_kv;
@@ -109,11 +117,14 @@ __host__ __device__ __forceinline__ int num_items(const AttnShape& sh) {
 
 // Epilogue of one query row: normalises its O (64 fp32 values read from
 // tensor memory), stores it as bf16 and writes lse = ln2 * (m*c + log2 l).
+// `c_log2` is the logits' scale in base 2 and `o_mul` a factor applied to O
+// (1 for bf16 inputs; the V dequantisation for e4m3 inputs).
 __device__ __forceinline__ void store_row(const uint32_t (&o)[64], int b, int h, int row, float m,
                                           float l, __nv_bfloat16* __restrict__ out,
-                                          float* __restrict__ lse, const AttnShape& sh) {
+                                          float* __restrict__ lse, const AttnShape& sh,
+                                          float c_log2, float o_mul) {
   if (row >= sh.T) return;
-  const float inv_l = 1.f / l;
+  const float inv_l = o_mul / l;
   uint4* dst = reinterpret_cast<uint4*>(out + ((static_cast<size_t>(b) * sh.T + row) * sh.H + h) * kD);
 #pragma unroll
   for (int v = 0; v < 8; ++v) {
@@ -125,15 +136,25 @@ __device__ __forceinline__ void store_row(const uint32_t (&o)[64], int b, int h,
     dst[v] = w;
   }
   lse[(static_cast<size_t>(b) * sh.H + h) * sh.T + row] =
-      (m * sh.scale_log2 + lg2(l)) * 0.69314718055994531f;
+      (m * c_log2 + lg2(l)) * 0.69314718055994531f;
 }
 
+// kFp8 = false: qkv is bf16, map_qkv covers it (128-byte swizzle) and map_v8
+// and dequant are unused. kFp8 = true: qkv holds e4m3 bytes; map_qkv covers
+// it with the 64-byte swizzle (Q and K tiles), map_v8 without swizzle (V
+// tiles, for the converter), and dequant[0..2] are the q, k, v dequantisation
+// multipliers. S = Q K^T then multiplies e4m3 operands (kind::f8f6f4) and the
+// softmax scale absorbs dequant[0] * dequant[1]; V becomes fp16 holding
+// e4m3 * 2^-8 exactly, and O is multiplied by 2^8 * dequant[2] at the end.
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __restrict__ out,
-                float* __restrict__ lse, const AttnShape sh) {
+attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
+                const __grid_constant__ CUtensorMap map_v8, __nv_bfloat16* __restrict__ out,
+                float* __restrict__ lse, const AttnShape sh, const float* __restrict__ dequant) {
+  constexpr int kQK = kQKBytes<kFp8>;
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                      ~uintptr_t(1023));
+  Smem<kFp8>& sm = *reinterpret_cast<Smem<kFp8>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int C = sh.H * kD;
@@ -161,7 +182,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == kProducerWarp && lane == 0) tma_prefetch_desc(&map_qkv);
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&map_qkv);
+    if (kFp8) tma_prefetch_desc(&map_v8);
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -182,7 +206,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         const Item it = decode_item(k, sh);
         const int slot = it_cnt & 1;
         if (!mbar_wait(&sm.q_empty[slot], ((it_cnt >> 1) & 1) ^ 1, kSiteFwdProducer, abort)) break;
-        mbar_arrive_expect_tx(&sm.q_full[slot], (it.has1 ? 2 : 1) * kTileBytes);
+        mbar_arrive_expect_tx(&sm.q_full[slot], (it.has1 ? 2 : 1) * kQK);
         tma_load_3d(sm.q[slot][0], &map_qkv, &sm.q_full[slot], it.h * kD, it.i0 * kBlockM, it.b);
         if (it.has1)
           tma_load_3d(sm.q[slot][1], &map_qkv, &sm.q_full[slot], it.h * kD,
@@ -195,9 +219,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kTileBytes);
+          mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kQK);
           tma_load_3d(sm.k[s], &map_qkv, &sm.kv_full[s], C + it.h * kD, j * kBlockN, it.b);
-          tma_load_3d(sm.v[s], &map_qkv, &sm.kv_full[s], 2 * C + it.h * kD, j * kBlockN, it.b);
+          if (kFp8)
+            tma_load_3d(sm.v8[s], &map_v8, &sm.kv_full[s], 2 * C + it.h * kD, j * kBlockN, it.b);
+          else
+            tma_load_3d(sm.v[s], &map_qkv, &sm.kv_full[s], 2 * C + it.h * kD, j * kBlockN, it.b);
         }
         if (!ok) break;
       }
@@ -219,6 +246,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
     const int q = warp - kMmaWarp;
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_s8 = idesc_e4m3_f32(128, 128);
       constexpr uint32_t idesc_o = idesc_f16_f32(128, 64, 0, 1);
       const uint32_t t_s = tmem + col_s(q), t_p = tmem + col_p(q), t_o = tmem + col_o(q);
       uint32_t kv_it = 0, it_cnt = 0, s_cnt = 0, p_cnt = 0;
@@ -247,18 +275,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         } else {
           if (!mbar_wait(&sm.q_full[slot], (it_cnt >> 1) & 1, kSiteFwdMma, abort)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.q[slot][q]), 16, 1024);
-          // S_q(jj) = Q_q K(jj)^T, K = 64 in steps of 16 (32 bytes).
+          const uint64_t qdesc = kFp8 ? smem_desc_sw64(smem_u32(sm.q[slot][q]), 512)
+                                      : smem_desc_sw128(smem_u32(sm.q[slot][q]), 16, 1024);
+          // S_q(jj) = Q_q K(jj)^T. bf16: K = 64 in four steps of 16 (32 bytes
+          // each); e4m3: two steps of 32 (32 bytes each).
           auto issue_s = [&](int jj) -> bool {
             const uint32_t idx = kv_it + jj;
             const int st = idx % kStages;
             if (!mbar_wait(&sm.kv_full[st], (idx / kStages) & 1, kSiteFwdMma, abort)) return false;
             if (s_cnt > 0 && !mbar_wait(&sm.s_free[q], (s_cnt - 1) & 1, kSiteFwdMma, abort)) return false;
             tc_fence_after();
-            const uint64_t kdesc = smem_desc_sw128(smem_u32(sm.k[st]), 16, 1024);
-            mma_ss(t_s, qdesc, kdesc, idesc_s, 0u);
+            if (kFp8) {
+              const uint64_t kdesc = smem_desc_sw64(smem_u32(sm.k[st]), 512);
+              mma_ss_f8(t_s, qdesc, kdesc, idesc_s8, 0u);
+              mma_ss_f8(t_s, qdesc + 2, kdesc + 2, idesc_s8, 1u);
+            } else {
+              const uint64_t kdesc = smem_desc_sw128(smem_u32(sm.k[st]), 16, 1024);
+              mma_ss(t_s, qdesc, kdesc, idesc_s, 0u);
 #pragma unroll
-            for (int kk = 1; kk < kD / 16; ++kk) mma_ss(t_s, qdesc + 2 * kk, kdesc + 2 * kk, idesc_s, 1u);
+              for (int kk = 1; kk < kD / 16; ++kk) mma_ss(t_s, qdesc + 2 * kk, kdesc + 2 * kk, idesc_s, 1u);
+            }
             mma_commit(&sm.s_full[q]);
             ++s_cnt;
             return true;
@@ -309,26 +345,48 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         ok = mbar_wait(&sm.kv_full[s], (kv_it / kStages) & 1, kSiteFwdConvert, abort);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        uint4* tile = reinterpret_cast<uint4*>(sm.v[s]);
-        // Running max of |v| over the converted fp16 values: a bf16 beyond
-        // fp16's range rounds to inf, so inf or NaN here flags the tile.
-        uint32_t mag = 0;
-#pragma unroll 4
-        for (int c = lane; c < kTileBytes / 16; c += 32) {
-          uint4 w = tile[c];
-          uint32_t* u = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            // bf16 -> fp32 is exact (a shift); fp32 -> fp16 rounds to nearest,
-            // exact for every bf16 value with |v| <= 65504 except fp16
-            // subnormals (|v| < 6.1e-5, within 3e-8).
-            u[e] = pack_f16(__uint_as_float(u[e] << 16), __uint_as_float(u[e] & 0xFFFF0000u));
-            mag = max_abs_f16x2(mag, u[e]);
+        if (kFp8) {
+          // e4m3 rows of 64 bytes, unswizzled, to fp16 rows of 128 bytes in
+          // the 128-byte swizzle: the 16 e4m3 values of input chunk c of row
+          // r fill fp16 chunks 2c and 2c + 1, stored at (chunk ^ (r & 7)).
+#pragma unroll 2
+          for (int idx = lane; idx < kTileBytes / 32; idx += 32) {
+            const int rr = idx >> 2, c = idx & 3;
+            const uint4 in = *reinterpret_cast<const uint4*>(sm.v8[s] + rr * 64 + c * 16);
+            const uint4 lo = make_uint4(e4m3x2_to_f16x2_scaled(in.x, 0x4140u),
+                                        e4m3x2_to_f16x2_scaled(in.x, 0x4342u),
+                                        e4m3x2_to_f16x2_scaled(in.y, 0x4140u),
+                                        e4m3x2_to_f16x2_scaled(in.y, 0x4342u));
+            const uint4 hi = make_uint4(e4m3x2_to_f16x2_scaled(in.z, 0x4140u),
+                                        e4m3x2_to_f16x2_scaled(in.z, 0x4342u),
+                                        e4m3x2_to_f16x2_scaled(in.w, 0x4140u),
+                                        e4m3x2_to_f16x2_scaled(in.w, 0x4342u));
+            uint8_t* row = sm.v[s] + rr * 128;
+            *reinterpret_cast<uint4*>(row + (((2 * c) ^ (rr & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ (rr & 7)) << 4)) = hi;
           }
-          tile[c] = w;
+        } else {
+          uint4* tile = reinterpret_cast<uint4*>(sm.v[s]);
+          // Running max of |v| over the converted fp16 values: a bf16 beyond
+          // fp16's range rounds to inf, so inf or NaN here flags the tile.
+          uint32_t mag = 0;
+#pragma unroll 4
+          for (int c = lane; c < kTileBytes / 16; c += 32) {
+            uint4 w = tile[c];
+            uint32_t* u = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              // bf16 -> fp32 is exact (a shift); fp32 -> fp16 rounds to
+              // nearest, exact for every bf16 value with |v| <= 65504 except
+              // fp16 subnormals (|v| < 6.1e-5, within 3e-8).
+              u[e] = pack_f16(__uint_as_float(u[e] << 16), __uint_as_float(u[e] & 0xFFFF0000u));
+              mag = max_abs_f16x2(mag, u[e]);
+            }
+            tile[c] = w;
+          }
+          if ((mag & 0x7FFFu) >= kF16InfBits || ((mag >> 16) & 0x7FFFu) >= kF16InfBits)
+            record_failure(kFwdValueRange);
         }
-        if ((mag & 0x7FFFu) >= kF16InfBits || ((mag >> 16) & 0x7FFFu) >= kF16InfBits)
-          record_failure(kFwdValueRange);
         // Generic-proxy stores must be visible to the tensor core (async proxy).
         fence_proxy_async_smem();
         __syncwarp();
@@ -339,6 +397,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
   } else {
     regs_alloc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
+    // The logits' scale in base 2, and the factor O is multiplied with at the
+    // end (both fold in the dequantisation of e4m3 inputs).
+    const float c_log2 = kFp8 ? sh.scale_log2 * dequant[0] * dequant[1] : sh.scale_log2;
+    const float o_mul = kFp8 ? 256.f * dequant[2] : 1.f;
     const int q = warp >> 2;                       // query tile of the pair
     const int r = ((warp & 3) << 5) + lane;        // row within the tile = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
@@ -362,7 +424,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
       const int i = it.i0 + q;
       const int row = i * kBlockM + r;
       // Running max m (raw logit units, as read from S) and running sum l of
-      // 2^(s*c - m*c), c = scale*log2(e). m is only raised when the row max
+      // 2^(s*c - m*c), c = c_log2. m is only raised when the row max
       // grows by more than kRescaleLog2 in log2 units; until then P and l keep
       // using the stale m, which stays exact because O / l uses the same m.
       float m = -INFINITY, l = 0.f;
@@ -402,10 +464,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[120 + e]);
         const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
                                fmaxf(mx8[6], mx8[7]));
-        const bool grow = (mx - m) * sh.scale_log2 > kRescaleLog2;  // always true on j == 0
+        const bool grow = (mx - m) * c_log2 > kRescaleLog2;  // always true on j == 0
         const float m_new = grow ? mx : m;
-        const float alpha = grow ? ex2((m - m_new) * sh.scale_log2) : 1.f;
-        const float neg_mc = -m_new * sh.scale_log2;
+        const float alpha = grow ? ex2((m - m_new) * c_log2) : 1.f;
+        const float neg_mc = -m_new * c_log2;
+        const bool flush = (j == 0) && pending;
+        // The FP8 forward keeps two more values live through the loop below
+        // (the runtime logit scale and output factor), so it waits for the
+        // previous P V product first and stores each half of P as soon as it
+        // is packed, holding 32 packed registers instead of 64.
+        constexpr bool kEarlyWait = kFp8;
+        if (kEarlyWait && (j > 0 || flush)) {
+          ok = mbar_wait(&sm.o_done[q], o_cnt & 1, kSiteFwdSoftmax, abort);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ++o_cnt;
+          tc_fence_after();
+        }
         // p = 2^(s*c - m*c), row sum, and fp16 packing of P in one pass. Every
         // kPolyEvery-th pair is exponentiated on the FMA pipe (exp2_poly2), the
         // rest on the exp unit, whose 16/clk rate bounds this loop otherwise.
@@ -414,7 +489,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
 #pragma unroll
         for (int c2 = 0; c2 < 64; ++c2) {
           float y0, y1, p0, p1;
-          fma2(x[2 * c2], x[2 * c2 + 1], sh.scale_log2, neg_mc, y0, y1);
+          fma2(x[2 * c2], x[2 * c2 + 1], c_log2, neg_mc, y0, y1);
           if (c2 % kPolyEvery == kPolyEvery - 1) {
             exp2_poly2(y0, y1, p0, p1);
           } else {
@@ -423,13 +498,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
           }
           add2(sa[c2 & 3], sb[c2 & 3], p0, p1);
           pk[c2] = pack_f16_nonneg(p0, p1);
+          if (kEarlyWait && c2 == 31) tmem_st32(t_p, *reinterpret_cast<uint32_t(*)[32]>(pk));
         }
         const float sum = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
         l = l * alpha + sum;
         m = m_new;
 
-        const bool flush = (j == 0) && pending;
-        if (j > 0 || flush) {
+        if (!kEarlyWait && (j > 0 || flush)) {
           // O must hold P_{j-1} V_{j-1} (or the finished item's last product)
           // before it is rescaled or read, and before P is reused.
           ok = mbar_wait(&sm.o_done[q], o_cnt & 1, kSiteFwdSoftmax, abort);
@@ -438,7 +513,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
           ++o_cnt;
           tc_fence_after();
         }
-        tmem_st32(t_p, *reinterpret_cast<uint32_t(*)[32]>(pk));
+        if (!kEarlyWait) tmem_st32(t_p, *reinterpret_cast<uint32_t(*)[32]>(pk));
         tmem_st32(t_p + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
         if (flush) {
           // The finished item's O is read before this tile's P V product (which
@@ -451,7 +526,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.p_full[q]);
-          store_row(o, p_b, p_h, p_row, p_m, p_l, out, lse, sh);
+          store_row(o, p_b, p_h, p_row, p_m, p_l, out, lse, sh, c_log2, o_mul);
           pending = false;
         } else {
           if (j > 0 && __any_sync(0xffffffffu, grow)) {
@@ -490,7 +565,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv, __nv_bfloat16* __re
         tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
         tmem_wait_ld();
         tc_fence_before();
-        store_row(o, p_b, p_h, p_row, p_m, p_l, out, lse, sh);
+        store_row(o, p_b, p_h, p_row, p_m, p_l, out, lse, sh, c_log2, o_mul);
       }
     }
   }

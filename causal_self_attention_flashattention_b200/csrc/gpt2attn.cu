@@ -4,8 +4,9 @@
 //
 // Nothing here allocates device memory. The only process-wide state is a
 // per-device cache of the SM count and of the kernels' shared-memory opt-in,
-// guarded by a mutex, the device status word the kernels write when a bounded
-// wait gives up, and the code of the last failed CUDA call.
+// guarded by a mutex, a cache of encoded tensor maps (its own mutex), the
+// device status word the kernels write when a bounded wait gives up, and the
+// code of the last failed CUDA call.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -25,6 +26,8 @@
 #include "bwd_fused.cuh"
 #include "decode.cuh"
 #include "selftest.cuh"
+#include "linear.cuh"
+#include "fp8.cuh"
 
 namespace ga_host {
 
@@ -94,14 +97,22 @@ const DeviceInfo* setup_device(int dev) {
   }
   if (cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return nullptr;
-  if (cudaFuncSetAttribute(ga::fwd::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(ga::fwd::kSmemBytes)) != cudaSuccess)
+  if (cudaFuncSetAttribute(ga::fwd::attn_fwd_kernel<false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::fwd::kSmemBytes<false>)) != cudaSuccess)
+    return nullptr;
+  if (cudaFuncSetAttribute(ga::fwd::attn_fwd_kernel<true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::fwd::kSmemBytes<true>)) != cudaSuccess)
     return nullptr;
   // The forward kernel's setmaxnreg split (warpgroup budgets that add up to the
   // block's allocation) is only safe if it launches with the register count
   // the split was sized for.
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel) != cudaSuccess ||
+  if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel<false>) != cudaSuccess ||
+      fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
+    return nullptr;
+  if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel<true>) != cudaSuccess ||
       fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
     return nullptr;
 
@@ -112,6 +123,9 @@ const DeviceInfo* setup_device(int dev) {
   if (cudaFuncSetAttribute(ga::bwd::fused::attn_bwd_fused_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(ga::bwd::fused::kSmemBytes)) != cudaSuccess)
+    return nullptr;
+  if (cudaFuncSetAttribute(ga::linear::linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::linear::kSmemBytes)) != cudaSuccess)
     return nullptr;
   if (cudaFuncSetAttribute(ga::bwd::dq::attn_bwd_dq_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -156,19 +170,108 @@ const DeviceInfo* device_info() {
   return ready;
 }
 
+// Tensor maps are cached: a map is a pure function of its description (base
+// address, data type, extents, box, swizzle), so a call that describes the
+// same tensor as an earlier one reuses the earlier encoding instead of asking
+// the driver again. The cache is a fixed table replaced round-robin under its
+// own mutex; it allocates nothing.
+struct MapKey {
+  const void* base;
+  uint64_t dims[3];
+  uint32_t box[3];
+  int rank, dtype, swizzle;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && dims[0] == o.dims[0] && dims[1] == o.dims[1] &&
+           dims[2] == o.dims[2] && box[0] == o.box[0] && box[1] == o.box[1] &&
+           box[2] == o.box[2] && rank == o.rank && dtype == o.dtype && swizzle == o.swizzle;
+  }
+};
+
+constexpr int kMapCacheSize = 64;
+struct MapCacheEntry {
+  bool used = false;
+  MapKey key;
+  CUtensorMap map;
+};
+std::mutex g_map_mutex;
+MapCacheEntry g_map_cache[kMapCacheSize];
+int g_map_next = 0;
+
+// Row-major tensor of `rank` <= 3 dims (innermost first) with `elem` bytes per
+// element and no padding between rows; box {box[0..rank)}; zero fill past
+// the edges. Returns false (recording the driver's code) if encoding fails.
+bool encode_map(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint32_t elem,
+                int rank, const uint64_t (&dims)[3], const uint32_t (&box)[3],
+                CUtensorMapSwizzle swizzle) {
+  MapKey key;
+  key.base = base;
+  key.rank = rank;
+  key.dtype = static_cast<int>(dtype);
+  key.swizzle = static_cast<int>(swizzle);
+  for (int d = 0; d < 3; ++d) {
+    key.dims[d] = d < rank ? dims[d] : 0;
+    key.box[d] = d < rank ? box[d] : 0;
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    for (const MapCacheEntry& e : g_map_cache)
+      if (e.used && e.key == key) {
+        *map = e.map;
+        return true;
+      }
+  }
+  cuuint64_t gdims[3], strides[2];
+  cuuint32_t gbox[3], elem_strides[3] = {1, 1, 1};
+  uint64_t stride = elem;
+  for (int d = 0; d < rank; ++d) {
+    gdims[d] = dims[d];
+    gbox[d] = box[d];
+    if (d > 0) strides[d - 1] = stride;
+    stride *= dims[d];
+  }
+  const CUresult r = g_encode(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
+                              gdims, strides, gbox, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    record_cuda_error(kCudaErrTensorMap, static_cast<unsigned int>(r));
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(g_map_mutex);
+  MapCacheEntry& e = g_map_cache[g_map_next];
+  g_map_next = (g_map_next + 1) % kMapCacheSize;
+  e.used = true;
+  e.key = key;
+  e.map = *map;
+  return true;
+}
+
 // 3-D bf16 tensor map {inner, T, B} with a {64, 128, 1} box, 128-byte swizzle
 // and zero fill outside the tensor (rows past T read as 0).
 bool make_map(CUtensorMap* map, const void* base, uint64_t inner, int T, int B) {
-  const cuuint64_t dims[3] = {inner, static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[2] = {inner * 2, inner * 2 * static_cast<cuuint64_t>(T)};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), static_cast<cuuint32_t>(ga::kBlockM), 1};
-  const cuuint32_t elem_strides[3] = {1, 1, 1};
-  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
-                              dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) record_cuda_error(kCudaErrTensorMap, static_cast<unsigned int>(r));
-  return r == CUDA_SUCCESS;
+  const uint64_t dims[3] = {inner, static_cast<uint64_t>(T), static_cast<uint64_t>(B)};
+  const uint32_t box[3] = {static_cast<uint32_t>(kD), static_cast<uint32_t>(ga::kBlockM), 1};
+  return encode_map(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3, dims, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// 3-D byte tensor map {inner, T, B} (e4m3 data) with a {64, 128, 1} box (64
+// bytes by 128 rows), the given swizzle and zero fill past the edges.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, int T, int B,
+                 CUtensorMapSwizzle swizzle) {
+  const uint64_t dims[3] = {inner, static_cast<uint64_t>(T), static_cast<uint64_t>(B)};
+  const uint32_t box[3] = {64, static_cast<uint32_t>(ga::kBlockM), 1};
+  return encode_map(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 3, dims, box, swizzle);
+}
+
+// 2-D bf16 tensor map {inner, rows} (row-major, `inner` contiguous) with a
+// {64, box_rows} box, 128-byte swizzle and zero fill past the edges.
+bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                 uint32_t box_rows) {
+  const uint64_t dims[3] = {inner, rows, 0};
+  const uint32_t box[3] = {64, box_rows, 0};
+  return encode_map(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2, dims, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // After a launch: GA_OK, or GA_ERR_CUDA with the launch error recorded.
@@ -219,9 +322,56 @@ ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse, int B, int T, in
   const ga::AttnShape sh = make_shape(B, T, H, scale);
   const int items = ga::fwd::num_items(sh);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  ga::fwd::attn_fwd_kernel<<<grid_for(items, info->num_sms), ga::fwd::kThreads,
-                             ga::fwd::kSmemBytes, s>>>(
-      map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh);
+  ga::fwd::attn_fwd_kernel<false><<<grid_for(items, info->num_sms), ga::fwd::kThreads,
+                                    ga::fwd::kSmemBytes<false>, s>>>(
+      map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr);
+  return check_launch();
+}
+
+ga_status gpt2_attn_fp8_quantize(const void* qkv, void* qkv8, float* scales, int B, int T, int H,
+                                 int D, gpt2attn_stream_t stream) {
+  if (qkv == nullptr || qkv8 == nullptr || scales == nullptr) return GA_ERR_INVALID_ARG;
+  const ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if (!aligned16(qkv) || !aligned16(qkv8) || !aligned16(scales)) return GA_ERR_ALIGNMENT;
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GA_ERR_CUDA;
+  const int C = H * kD;
+  const long long n_chunks = static_cast<long long>(B) * T * 3 * C / 8;
+  const long long want = (n_chunks + ga::fp8::kThreads - 1) / ga::fp8::kThreads;
+  const long long cap = 8LL * info->num_sms;
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ga::fp8::fp8_zero_kernel<<<1, 32, 0, s>>>(scales);
+  ga::fp8::fp8_amax_kernel<<<blocks, ga::fp8::kThreads, 0, s>>>(
+      static_cast<const uint4*>(qkv), n_chunks, C, scales);
+  ga::fp8::fp8_quantize_kernel<<<blocks, ga::fp8::kThreads, 0, s>>>(
+      static_cast<const uint4*>(qkv), static_cast<uint2*>(qkv8), n_chunks, C, scales);
+  return check_launch();
+}
+
+ga_status gpt2_attn_fwd_fp8(const void* qkv8, const float* scales, void* out, float* lse, int B,
+                            int T, int H, int D, float scale, gpt2attn_stream_t stream) {
+  if (qkv8 == nullptr || scales == nullptr || out == nullptr || lse == nullptr)
+    return GA_ERR_INVALID_ARG;
+  ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if ((st = check_scale(scale)) != GA_OK) return st;
+  if (!aligned16(qkv8) || !aligned16(scales) || !aligned16(out) || !aligned16(lse))
+    return GA_ERR_ALIGNMENT;
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GA_ERR_CUDA;
+  CUtensorMap map_qk, map_v;
+  const uint64_t inner = static_cast<uint64_t>(3) * H * kD;
+  if (!make_map_u8(&map_qk, qkv8, inner, T, B, CU_TENSOR_MAP_SWIZZLE_64B)) return GA_ERR_CUDA;
+  if (!make_map_u8(&map_v, qkv8, inner, T, B, CU_TENSOR_MAP_SWIZZLE_NONE)) return GA_ERR_CUDA;
+  const ga::AttnShape sh = make_shape(B, T, H, scale);
+  const int items = ga::fwd::num_items(sh);
+  ga::fwd::attn_fwd_kernel<true><<<grid_for(items, info->num_sms), ga::fwd::kThreads,
+                                   ga::fwd::kSmemBytes<true>,
+                                   reinterpret_cast<cudaStream_t>(stream)>>>(
+      map_qk, map_v, static_cast<__nv_bfloat16*>(out), lse, sh,
+      scales + ga::fp8::kDequantOffset);
   return check_launch();
 }
 
@@ -412,6 +562,62 @@ ga_status gpt2_attn_decode(const void* qkv, int t, void* out, float* lse, void* 
   ga::decode::attn_decode_combine_kernel<<<dim3(H, B), ga::kD, 0, s>>>(
       partials, n_chunks, static_cast<__nv_bfloat16*>(out), lse, sh);
   return check_launch();
+}
+
+namespace {
+
+// y (M, N) = a (M, K) w (N, K)^T + bias (N): the shared body of the two dense
+// layers. K and N are multiples of 64 here (C = H * 64).
+ga_status launch_linear(const void* a, const void* w, const void* bias, void* y, long long M,
+                        int N, int K, gpt2attn_stream_t stream) {
+  if (static_cast<long double>(M) * (N > K ? N : K) >= 2147483648.0L) return GA_ERR_INVALID_ARG;
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GA_ERR_CUDA;
+  CUtensorMap map_a, map_w;
+  if (!make_map_2d(&map_a, a, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                   ga::linear::kBM))
+    return GA_ERR_CUDA;
+  if (!make_map_2d(&map_w, w, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                   ga::linear::kBN))
+    return GA_ERR_CUDA;
+  ga::linear::GemmShape g;
+  g.M = static_cast<int>(M);
+  g.N = N;
+  g.K = K;
+  g.tiles_n = ga::ceil_div(N, ga::linear::kBN);
+  g.f16_from = N;
+  const int tiles = ga::ceil_div(g.M, ga::linear::kBM) * g.tiles_n;
+  ga::linear::linear_kernel<<<grid_for(tiles, info->num_sms), ga::linear::kThreads,
+                              ga::linear::kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(
+      map_a, map_w, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(y), g);
+  return check_launch();
+}
+
+ga_status check_linear_args(const void* a, const void* w, const void* bias, const void* y, int B,
+                            int T, int H, int D) {
+  if (a == nullptr || w == nullptr || bias == nullptr || y == nullptr) return GA_ERR_INVALID_ARG;
+  const ga_status st = check_shape(B, T, H, D);
+  if (st != GA_OK) return st;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(bias) || !aligned16(y)) return GA_ERR_ALIGNMENT;
+  return GA_OK;
+}
+
+}  // namespace
+
+ga_status gpt2_attn_qkv_proj(const void* x, const void* w_attn, const void* b_attn, void* qkv,
+                             int B, int T, int H, int D, gpt2attn_stream_t stream) {
+  const ga_status st = check_linear_args(x, w_attn, b_attn, qkv, B, T, H, D);
+  if (st != GA_OK) return st;
+  const int C = H * D;
+  return launch_linear(x, w_attn, b_attn, qkv, static_cast<long long>(B) * T, 3 * C, C, stream);
+}
+
+ga_status gpt2_attn_out_proj(const void* out, const void* w_proj, const void* b_proj, void* y,
+                             int B, int T, int H, int D, gpt2attn_stream_t stream) {
+  const ga_status st = check_linear_args(out, w_proj, b_proj, y, B, T, H, D);
+  if (st != GA_OK) return st;
+  const int C = H * D;
+  return launch_linear(out, w_proj, b_proj, y, static_cast<long long>(B) * T, C, C, stream);
 }
 
 ga_status gpt2_attn_selftest_wait_timeout(unsigned long long limit_ns, gpt2attn_stream_t stream) {

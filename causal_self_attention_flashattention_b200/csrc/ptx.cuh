@@ -158,6 +158,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// 2-D tiled load of one box into shared memory (same completion mechanism).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor-core MMA
 // ---------------------------------------------------------------------------
@@ -202,6 +212,18 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem] with 8-bit (e4m3) operands: 32 elements of K
+// per instruction.
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -304,6 +326,25 @@ __device__ __forceinline__ uint64_t smem_desc_noswizzle(uint32_t saddr, uint32_t
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= 1ull << 46;
   return d;
+}
+
+// Shared-memory descriptor for a K-major tile with 64-byte rows and the
+// 64-byte swizzle (8-row atoms 512 bytes apart), as TMA writes a box whose
+// inner extent is 64 bytes: swizzle mode 4 in [61,64), otherwise as above.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 4ull << 61;
+  return d;
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format code 0)
+// and fp32 accumulate, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor for kind::f16 with bf16 inputs and fp32 accumulate.
@@ -511,6 +552,28 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u, uint32_t& rng) {
   rng = max_u16x2(rng, mag);
   const uint32_t clamped = max_u16x2(mag, 0x38003800u);
   return (clamped * 8u + 0x3FFE4000u) | (u & 0x80008000u);
+}
+
+// Two e4m3 values (bytes 0 and 1, or 2 and 3, of `w`, picked by `sel`) as an
+// fp16 pair equal to the e4m3 values times 2^-8, with integer operations
+// only. An e4m3 byte s.eeee.mmm (exponent bias 7) becomes the fp16 bits
+// s.0eeee.mmm0000000 (exponent bias 15): the exponent field keeps its value,
+// so every value, subnormals included, is scaled by exactly 2^(7-15). The
+// sign moves from bit 7 to bit 8 of the 16-bit lane by adding the byte's own
+// top bit to it (no carry leaves the lane), then the lane shifts by 7.
+// `sel` is 0x4140 for bytes 0, 1 and 0x4342 for bytes 2, 3.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t sel) {
+  uint32_t t;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(t) : "r"(w), "r"(sel));
+  return (t + (t & 0x00800080u)) << 7;
+}
+
+// Two floats to an e4m3 pair (round to nearest even, saturating to +-448);
+// `lo` goes to the low byte.
+__device__ __forceinline__ uint16_t pack_e4m3(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Warpgroup-wide register budget changes (all four warps of a warpgroup

@@ -49,6 +49,10 @@ EXPORTED_SYMBOLS = (
     "gpt2_attn_decode",
     "gpt2_attn_last_device_status",
     "gpt2_attn_selftest_wait_timeout",
+    "gpt2_attn_qkv_proj",
+    "gpt2_attn_fp8_quantize",
+    "gpt2_attn_fwd_fp8",
+    "gpt2_attn_out_proj",
     "gpt2_attn_status_string",
     "gpt2_attn_version",
 )
@@ -88,6 +92,14 @@ _lib.gpt2_attn_decode.argtypes = [_vp, _i, _vp, _vp, _vp, ctypes.c_size_t, _i, _
 _lib.gpt2_attn_decode.restype = _i
 _lib.gpt2_attn_last_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
 _lib.gpt2_attn_last_device_status.restype = _i
+_lib.gpt2_attn_fp8_quantize.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp]
+_lib.gpt2_attn_fp8_quantize.restype = _i
+_lib.gpt2_attn_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_fwd_fp8.restype = _i
+_lib.gpt2_attn_qkv_proj.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+_lib.gpt2_attn_qkv_proj.restype = _i
+_lib.gpt2_attn_out_proj.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+_lib.gpt2_attn_out_proj.restype = _i
 _lib.gpt2_attn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, _vp]
 _lib.gpt2_attn_selftest_wait_timeout.restype = _i
 _lib.gpt2_attn_status_string.argtypes = [_i]
@@ -388,3 +400,84 @@ class CausalSelfAttention(torch.autograd.Function):
 def causal_self_attention(qkv: torch.Tensor, scale: float | None = None) -> torch.Tensor:
     """One-call causal self-attention on packed qkv (B,T,3,H,D) -> (B,T,H,D)."""
     return CausalSelfAttention.apply(qkv, scale)
+
+
+def qkv_proj(x: torch.Tensor, w_attn: torch.Tensor, b_attn: torch.Tensor, H: int,
+             qkv: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """c_attn: qkv = x W_attn^T + b_attn, returned as packed (B, T, 3, H, D) bf16.
+
+    x (B, T, C) bf16, w_attn (3C, C) bf16 (nn.Linear layout), b_attn (3C,) bf16.
+    """
+    if x.dim() != 3:
+        raise ValueError(f"x must be (B, T, C), got {tuple(x.shape)}")
+    B, T, C = (int(d) for d in x.shape)
+    if C % H:
+        raise ValueError("C must be a multiple of H")
+    D = C // H
+    _expect(x, "x", (B, T, C), torch.bfloat16)
+    _expect(w_attn, "w_attn", (3 * C, C), torch.bfloat16)
+    _expect(b_attn, "b_attn", (3 * C,), torch.bfloat16)
+    if qkv is None:
+        qkv = torch.empty((B, T, 3, H, D), dtype=torch.bfloat16, device=x.device)
+    _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
+    _check(_lib.gpt2_attn_qkv_proj(x.data_ptr(), w_attn.data_ptr(), b_attn.data_ptr(),
+                                   qkv.data_ptr(), B, T, H, D, _stream_ptr(stream)),
+           "gpt2_attn_qkv_proj")
+    return qkv
+
+
+def out_proj(out: torch.Tensor, w_proj: torch.Tensor, b_proj: torch.Tensor,
+             y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """c_proj: y = out W_proj^T + b_proj from the attention output (B, T, H, D);
+    returns y (B, T, C) bf16. w_proj (C, C) bf16, b_proj (C,) bf16."""
+    if out.dim() != 4:
+        raise ValueError(f"out must be (B, T, H, D), got {tuple(out.shape)}")
+    B, T, H, D = (int(d) for d in out.shape)
+    C = H * D
+    _expect(out, "out", (B, T, H, D), torch.bfloat16)
+    _expect(w_proj, "w_proj", (C, C), torch.bfloat16)
+    _expect(b_proj, "b_proj", (C,), torch.bfloat16)
+    if y is None:
+        y = torch.empty((B, T, C), dtype=torch.bfloat16, device=out.device)
+    _expect(y, "y", (B, T, C), torch.bfloat16)
+    _check(_lib.gpt2_attn_out_proj(out.data_ptr(), w_proj.data_ptr(), b_proj.data_ptr(),
+                                   y.data_ptr(), B, T, H, D, _stream_ptr(stream)),
+           "gpt2_attn_out_proj")
+    return y
+
+
+def fp8_quantize(qkv: torch.Tensor, qkv8: torch.Tensor | None = None,
+                 scales: torch.Tensor | None = None, stream=None):
+    """Per-tensor e4m3 quantisation of q, k, v: returns (qkv8 (B,T,3,H,D)
+    uint8 e4m3 bytes, scales fp32[8] whose [0..2] are the dequantisation
+    multipliers)."""
+    B, T, H, D = _dims(qkv)
+    _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
+    if qkv8 is None:
+        qkv8 = torch.empty((B, T, 3, H, D), dtype=torch.uint8, device=qkv.device)
+    if scales is None:
+        scales = torch.empty(8, dtype=torch.float32, device=qkv.device)
+    _expect(qkv8, "qkv8", (B, T, 3, H, D), torch.uint8)
+    _expect(scales, "scales", (8,), torch.float32)
+    _check(_lib.gpt2_attn_fp8_quantize(qkv.data_ptr(), qkv8.data_ptr(), scales.data_ptr(),
+                                       B, T, H, D, _stream_ptr(stream)), "gpt2_attn_fp8_quantize")
+    return qkv8, scales
+
+
+def attn_fwd_fp8(qkv8: torch.Tensor, scales: torch.Tensor, scale: float | None = None,
+                 out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """FP8 forward from fp8_quantize's output: returns (out bf16, lse fp32)."""
+    B, T, H, D = _dims(qkv8)
+    _expect(qkv8, "qkv8", (B, T, 3, H, D), torch.uint8)
+    _expect(scales, "scales", (8,), torch.float32)
+    scale = default_scale(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=qkv8.device)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=qkv8.device)
+    _expect(out, "out", (B, T, H, D), torch.bfloat16)
+    _expect(lse, "lse", (B, H, T), torch.float32)
+    _check(_lib.gpt2_attn_fwd_fp8(qkv8.data_ptr(), scales.data_ptr(), out.data_ptr(),
+                                  lse.data_ptr(), B, T, H, D, scale, _stream_ptr(stream)),
+           "gpt2_attn_fwd_fp8")
+    return out, lse

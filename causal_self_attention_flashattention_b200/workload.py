@@ -26,7 +26,8 @@ from dataclasses import dataclass
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "attention_flops", "algorithmic_bytes"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_linear_inputs", "attention_flops",
+           "algorithmic_bytes"]
 
 
 @dataclass(frozen=True)
@@ -62,6 +63,19 @@ def make_inputs(B: int, T: int, H: int, D: int = 64, seed: int = 0, qk_std: floa
     if qk_std != 1.0:
         qkv[:, :, 0:2] *= qk_std
     return qkv.to(torch.bfloat16), dout.to(torch.bfloat16)
+
+
+def make_linear_inputs(B: int, T: int, C: int, n_out: int, seed: int = 0):
+    """Returns (x, w, b) for a dense layer C -> n_out as CPU bf16 tensors:
+    x (B, T, C) ~ N(0, 1) (the normalised activations a GPT-2 block feeds its
+    layers), w (n_out, C) and b (n_out,) ~ N(0, 0.02^2) (GPT-2's weight
+    initialisation scale; the bias is drawn too so that its addition is
+    exercised)."""
+    g = torch.Generator().manual_seed(int(seed))
+    x = torch.randn(B, T, C, dtype=torch.float32, generator=g)
+    w = torch.randn(n_out, C, dtype=torch.float32, generator=g) * 0.02
+    b = torch.randn(n_out, dtype=torch.float32, generator=g) * 0.02
+    return x.to(torch.bfloat16), w.to(torch.bfloat16), b.to(torch.bfloat16)
 
 
 def attention_flops(B: int, T: int, H: int, D: int) -> tuple[float, float]:

@@ -30,8 +30,10 @@
  *   - Every pointer must be non-null and 16-byte aligned.
  *   - scale must be finite and > 0; GPT-2 uses 1/sqrt(D) = 0.125.
  *   - The caller owns every buffer, including the backward workspace. The
- *     library allocates nothing per call and keeps no state between calls,
- *     apart from a device status word that records a timed-out wait.
+ *     library allocates nothing per call. Between calls it keeps only host
+ *     caches (per-device set-up and the TMA descriptors of recently seen
+ *     tensors, keyed by address, extents and layout, each behind a mutex) and
+ *     a device status word that records a timed-out wait.
  *   - Calls only enqueue work on `stream` (the legacy default stream when
  *     NULL). They never synchronise. Arguments are checked before anything is
  *     launched: on any error nothing is launched and the status says why.
@@ -72,10 +74,11 @@ typedef enum {
  * with fp32 accumulators in tensor memory, the online softmax runs in
  * registers, key tiles above the diagonal are skipped, and lse is written
  * per query row. S = Q K^T multiplies bf16 operands. O += P V multiplies
- * fp16 operands: P keeps 11 significant bits, and each bf16 v converts to
- * fp16 exactly when |v| <= 65504. A v entry with |v| above that, or an inf or
- * NaN, is reported as GA_ERR_RANGE by gpt2_attn_last_device_status; the
- * outputs of that call are then undefined.
+ * fp16 operands: P keeps 11 significant bits, and each bf16 v with
+ * 2^-14 <= |v| <= 65280 converts to fp16 exactly (smaller ones move by less
+ * than 2^-15). A v entry beyond fp16's range (|v| >= 65536, inf or NaN) is
+ * reported as GA_ERR_RANGE by gpt2_attn_last_device_status; the outputs of
+ * that call are then undefined.
  */
 ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse,
                         int B, int T, int H, int D, float scale,
@@ -219,6 +222,67 @@ ga_status gpt2_attn_bwd_noalloc(const void* qkv, const void* out, const void* do
                                 const float* lse, void* dqkv,
                                 int B, int T, int H, int D, float scale,
                                 gpt2attn_stream_t stream);
+
+/*
+ * FP8 forward: the attention of e4m3 q, k, v with one scale per tensor. The
+ * llm.c page plans FP8 training ("Réimplémenter à bas coût le modèle GPT-2
+ * avec llm.c", FAQ entry on FP8); the pages fix no format, so each of q, k
+ * and v gets the scale that maps its largest magnitude to 448, the largest
+ * e4m3 value. Results are those of the attention of the dequantised inputs
+ * (e4m3 value * dequant), not of the bf16 ones: the e4m3 rounding of the
+ * inputs moves the output far more than the bf16 path's error.
+ *
+ * gpt2_attn_fp8_quantize: qkv (bf16, as gpt2_attn_fwd reads it) to
+ *   qkv8  [out] e4m3 bytes (B,T,3,H,D), same layout, one byte per element
+ *   scales [out/scratch] fp32[8], device, 16-byte aligned: [0..2] receive the
+ *          dequantisation multipliers of q, k, v (amax / 448, or 1 for an
+ *          all-zero tensor); [4..6] are scratch (the amax words)
+ *   with amax = max |x| per slot, x8 = e4m3(x * (448 / amax)) rounded to
+ *   nearest even (every fp32 step correctly rounded). Three launches on
+ *   `stream`: clear the amax words, reduce amax, scale and round. NaN inputs
+ *   are skipped by the amax and stay NaN.
+ * gpt2_attn_fwd_fp8: out and lse from qkv8 and scales as written by
+ *   gpt2_attn_fp8_quantize (earlier on the same stream); out, lse and scale
+ *   as for gpt2_attn_fwd. S = Q K^T multiplies the e4m3 operands on the
+ *   tensor cores (kind::f8f6f4, fp32 accumulation); the softmax scale absorbs
+ *   dequant_q * dequant_k; V is widened to fp16 (exact) for O += P V, and O is
+ *   multiplied by dequant_v.
+ */
+ga_status gpt2_attn_fp8_quantize(const void* qkv, void* qkv8, float* scales,
+                                 int B, int T, int H, int D, gpt2attn_stream_t stream);
+ga_status gpt2_attn_fwd_fp8(const void* qkv8, const float* scales, void* out, float* lse,
+                            int B, int T, int H, int D, float scale,
+                            gpt2attn_stream_t stream);
+
+/*
+ * The two dense layers on either side of attention in a GPT-2 block
+ * ("Andrej Karpathy - Lets reproduce GPT 2 124M" video description, chapter
+ * 00:13:47, the GPT-2 nn.Module; "Comment recréer GPT2 en 4 heures ?",
+ * section 5, the rearranged blocks), on the tensor cores (bf16 inputs, fp32
+ * accumulation in tensor memory, bias added in fp32, one rounding to bf16).
+ * Weights use nn.Linear's layout (out_features, in_features), row-major.
+ * C = H * D with D == 64; B, T, H as for the attention calls; every pointer
+ * 16-byte aligned; B*T*3C below 2^31.
+ *
+ * gpt2_attn_qkv_proj (c_attn): qkv = x W_attn^T + b_attn
+ *   x      [in]  bf16 (B,T,C)
+ *   w_attn [in]  bf16 (3C, C)
+ *   b_attn [in]  bf16 (3C)
+ *   qkv    [out] bf16 (B,T,3,H,D): the row-major (B*T, 3C) result, which is
+ *                exactly the packed layout gpt2_attn_fwd reads
+ * gpt2_attn_out_proj (c_proj): y = out W_proj^T + b_proj
+ *   out    [in]  bf16 (B,T,H,D): gpt2_attn_fwd's output, read as (B*T, C)
+ *   w_proj [in]  bf16 (C, C)
+ *   b_proj [in]  bf16 (C)
+ *   y      [out] bf16 (B,T,C)
+ * One launch each on `stream`; inputs and outputs must not overlap.
+ */
+ga_status gpt2_attn_qkv_proj(const void* x, const void* w_attn, const void* b_attn,
+                             void* qkv, int B, int T, int H, int D,
+                             gpt2attn_stream_t stream);
+ga_status gpt2_attn_out_proj(const void* out, const void* w_proj, const void* b_proj,
+                             void* y, int B, int T, int H, int D,
+                             gpt2attn_stream_t stream);
 
 /*
  * Self-test of the device-side failure path that every kernel of this library

@@ -6,7 +6,7 @@ from bf16 inputs; per 128-key tile, the row max with the stale-max rule
 (raised only when it grows by more than 2^8 in base 2), p = 2^(s*c - m*c)
 with every 4th pair of columns on the FMA-pipe polynomial, the row sum in the
 kernel's order, P packed to fp16 (round half up) and multiplied with V
-converted to fp16, O rescaled when the max is raised; at the end
+converted to fp16 (the integer conversion: exact down to 2^-14), O rescaled when the max is raised; at the end
 out = bf16(O / l) and lse = ln2 * (m*c + log2 l). Replacing the fp16 P and V
 with bf16 shows what the precision choice buys.
 """
@@ -17,11 +17,24 @@ import pytest
 from oracle import oracle as orc
 from causal_self_attention_flashattention_b200.workload import make_inputs
 
-from .test_kernel_arith import _bf16_rne, exp2_poly_model, pack_f16_nonneg_model
+from .test_kernel_arith import (_bf16_rne, bf16x2_to_f16x2_model, exp2_poly_model,
+                                pack_f16_nonneg_model)
 from .test_parity_gpu import LSE_TOL, out_error_ok
 
 LOG2E = 1.4426950408889634
 POLY_COLS = np.array([(col // 2) % 4 == 3 for col in range(128)])
+
+
+def v_to_f16_model(V):
+    """V (bf16 values held in float32) as the forward's integer conversion
+    turns them into fp16, back in float32. Values that are not bf16 (the
+    dequantized e4m3 inputs below) are rounded to fp16 directly."""
+    bits = np.ascontiguousarray(V, dtype=np.float32).view(np.uint32)
+    if np.any(bits & np.uint32(0xFFFF)):
+        return np.asarray(V, np.float32).astype(np.float16).astype(np.float32)
+    r, _, _ = bf16x2_to_f16x2_model((bits >> np.uint32(16)).ravel())
+    h = (r & np.uint32(0xFFFF)).astype(np.uint16).view(np.float16)
+    return h.astype(np.float32).reshape(V.shape)
 
 
 def kernel_forward_model(Q, K, V, scale, p_format="f16"):
@@ -29,7 +42,7 @@ def kernel_forward_model(Q, K, V, scale, p_format="f16"):
     T, D = V.shape
     c = np.float32(np.float32(scale) * np.float32(LOG2E))
     S = (Q @ K.T).astype(np.float32)
-    Vp = V.astype(np.float16).astype(np.float32) if p_format == "f16" else V
+    Vp = v_to_f16_model(V) if p_format == "f16" else V
     m = np.full(T, -np.inf, np.float32)
     l = np.zeros(T, np.float32)
     O = np.zeros((T, D), np.float32)
@@ -241,3 +254,23 @@ def test_e4m3_inputs_move_the_result_beyond_the_tolerances():
     ok, err, _ = out_error_ok(out.astype(np.float64), Oq)
     assert ok, err
     assert np.max(np.abs(lse_m - lseq)) <= LSE_TOL
+
+
+def test_fp8_forward_model_rounds_faithfully_on_peaked_rows():
+    # The FP8 forward's arithmetic (exact e4m3 logits, fp16 P and V) on the
+    # dequantised stress inputs, head (0, 8): one output element near 4 lies
+    # about 2e-3 from the exact value in fp32 and rounds to the far bf16
+    # neighbour, so correct rounding fails while faithful rounding (either
+    # enclosing bf16 value) holds; lse stays far inside 1e-3.
+    from oracle import fp8 as ofp8
+    from .test_parity_gpu import out_error_ok, out_error_ok_faithful
+
+    qkv, _ = make_inputs(4, 4096, 12, 64, seed=0, qk_std=3.0)
+    bits, dq = ofp8.quantize_qkv(qkv.float().numpy())
+    deq = ofp8.dequantize_qkv(bits, dq)
+    Q, K, V = (deq[0, :, s, 8] for s in range(3))
+    O, lse, _ = orc.head_forward(Q, K, V, 0.125)
+    out, lse_m = kernel_forward_model(Q, K, V, 0.125, "f16")
+    assert not out_error_ok(out.astype(np.float64), O)[0]
+    assert out_error_ok_faithful(out.astype(np.float64), O)[0]
+    assert np.max(np.abs(lse_m - lse)) <= LSE_TOL
