@@ -601,7 +601,7 @@ def run_decode(args, wl):
         "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "B": B, "T": T, "H": H, "D": D, "t": t,
                    "l2": f"{len(sets)} rotating qkv buffers of {qkv_cpu.numel() * 2} B > 126 MB L2",
-                   "step": "gpt2_attn_decode (partial per 256-key chunk, then combine)"},
+                   "step": "gpt2_attn_decode (partial per 128-key chunk, TMA-staged, then combine)"},
         "roofline": {"kernel": "decode", "bound": "hbm", "achieved": gbs,
                      "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                      "frac": gbs / float(peaks["hbm_gbs"]), "peak_source": f"hbm_gbs of {peak_src}",

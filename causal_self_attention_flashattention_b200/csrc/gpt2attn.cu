@@ -557,8 +557,11 @@ ga_status gpt2_attn_decode(const void* qkv, int t, void* out, float* lse, void* 
   const int n_chunks = ga::decode::num_chunks(t);
   float* partials = static_cast<float*>(workspace);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  ga::decode::attn_decode_partial_kernel<<<dim3(n_chunks, H, B), ga::decode::kWarps * 32, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(qkv), t, partials, sh);
+  CUtensorMap map_qkv;
+  if (!make_map(&map_qkv, qkv, static_cast<uint64_t>(3) * H * kD, T, B)) return GA_ERR_CUDA;
+  ga::decode::attn_decode_partial_kernel<<<dim3(n_chunks, H, B), ga::decode::kWarps * 32,
+                                           ga::decode::kSmemBytes, s>>>(
+      map_qkv, static_cast<const __nv_bfloat16*>(qkv), t, partials, sh);
   ga::decode::attn_decode_combine_kernel<<<dim3(H, B), ga::kD, 0, s>>>(
       partials, n_chunks, static_cast<__nv_bfloat16*>(out), lse, sh);
   return check_launch();

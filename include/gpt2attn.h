@@ -186,9 +186,10 @@ ga_status gpt2_attn_bwd_fused(const void* qkv, const void* dout, const float* ls
  *   lse   [out] fp32 (B,H), device: natural log of sum_j exp(scale q.k_j)
  *   workspace [scratch] >= gpt2_attn_decode_workspace_size bytes, 16-byte
  *         aligned, not shared by calls that run concurrently
- * Two launches on `stream`: per 256-key chunk of each (b,h), partial max, sum
- * and unnormalised output (fp32, CUDA cores: the step is bound by reading k
- * and v); then one combine per (b,h). GA_ERR_INVALID_ARG for t outside
+ * Two launches on `stream`: per 128-key chunk of each (b,h), partial max, sum
+ * and unnormalised output (the chunk's k and v rows staged in shared memory
+ * by TMA; fp32 on the CUDA cores: the step is bound by reading k and v); then
+ * one combine per (b,h). GA_ERR_INVALID_ARG for t outside
  * [0, T) or B, H above 65535.
  */
 ga_status gpt2_attn_decode_workspace_size(int B, int T, int H, int D, size_t* bytes);

@@ -148,8 +148,8 @@ def test_decode_arguments_rejected_before_launch():
     p = 1 << 20  # a 16-byte-aligned fake address: nothing is launched on these paths
     n = ctypes.c_size_t(0)
     assert lib.gpt2_attn_decode_workspace_size(2, 1000, 3, 64, ctypes.byref(n)) == ops.GA_OK
-    # partials fp32 [B][H][ceil(T/256)][2 + D]
-    assert n.value == 2 * 3 * 4 * 66 * 4
+    # partials fp32 [B][H][ceil(T/128)][2 + D]
+    assert n.value == 2 * 3 * 8 * 66 * 4
     ws = n.value
     assert lib.gpt2_attn_decode(p, 1000, p, p, p, ws, 2, 1000, 3, 64, 0.125, None) == ops.GA_ERR_INVALID_ARG
     assert lib.gpt2_attn_decode(p, -1, p, p, p, ws, 2, 1000, 3, 64, 0.125, None) == ops.GA_ERR_INVALID_ARG
