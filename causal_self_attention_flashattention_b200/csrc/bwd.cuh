@@ -110,22 +110,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 // S^T - lse/scale and dP^T - Delta (one extra K step of each product adds the
 // per-query constants), so P^T = 2^(c x) (zero where the key r comes after
 // query c0 + e when kMasked) and dS^T = P^T o dP'^T, both packed to bf16 pairs.
-// One pair in kBwdPolyEvery (0: none) is exponentiated on the FMA pipe
-// (exp2_poly2) instead of the exp unit.
-constexpr int kBwdPolyEvery = 0;
-
-__device__ __forceinline__ void exp2_pair(int pair, float x0, float x1, float& p0, float& p1) {
-  if (kBwdPolyEvery > 0 && pair % (kBwdPolyEvery > 0 ? kBwdPolyEvery : 1) == kBwdPolyEvery - 1) {
-    exp2_poly2(x0, x1, p0, p1);
-    // The polynomial returns a tiny positive value instead of 0 for -inf.
-    p0 = x0 == -INFINITY ? 0.f : p0;
-    p1 = x1 == -INFINITY ? 0.f : p1;
-  } else {
-    p0 = ex2(x0);
-    p1 = ex2(x1);
-  }
-}
-
 template <bool kMasked>
 __device__ __forceinline__ void dkdv_chunk(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
                                            float sc, int c0, int r, uint32_t (&pp)[8],
@@ -138,8 +122,7 @@ __device__ __forceinline__ void dkdv_chunk(const uint32_t (&sv)[16], const uint3
       if (c0 + c < r) x0 = -INFINITY;
       if (c0 + c + 1 < r) x1 = -INFINITY;
     }
-    float p0, p1;
-    exp2_pair(c >> 1, x0, x1, p0, p1);
+    const float p0 = ex2(x0), p1 = ex2(x1);
     mul2v(p0, p1, __uint_as_float(dv[c]), __uint_as_float(dv[c + 1]), d0, d1);
     pp[c >> 1] = pack_bf16(p0, p1);
     dd[c >> 1] = pack_bf16(d0, d1);
@@ -161,8 +144,7 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[16], const uint32_
       if (c0 + c > r) x0 = -INFINITY;
       if (c0 + c + 1 > r) x1 = -INFINITY;
     }
-    float p0, p1;
-    exp2_pair(c >> 1, x0, x1, p0, p1);
+    const float p0 = ex2(x0), p1 = ex2(x1);
     float t0 = __uint_as_float(dv[c]), t1 = __uint_as_float(dv[c + 1]);
     add2(t0, t1, nd, nd);
     mul2v(p0, p1, t0, t1, d0, d1);
