@@ -52,6 +52,8 @@ WORKLOADS = {
     "gpt2-124m-b64-t1024": Workload("gpt2-124m-b64-t1024", 64, 1024, 12),
     "gpt2-350m-b32-t1024": Workload("gpt2-350m-b32-t1024", 32, 1024, 16),
     "stress-b4-t4096-qk3": Workload("stress-b4-t4096-qk3", 4, 4096, 12, qk_std=3.0),
+    # A quarter of the bench batch: the size the full ncu captures run at.
+    "gpt2-124m-b4-t1024": Workload("gpt2-124m-b4-t1024", 4, 1024, 12),
 }
 
 
