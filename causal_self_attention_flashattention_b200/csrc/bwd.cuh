@@ -215,7 +215,10 @@ __device__ __forceinline__ uint32_t bf16_pair(__nv_bfloat16 lo, __nv_bfloat16 hi
 }
 
 struct alignas(1024) Smem {
-  uint8_t k[2][kTileBytes];  // [item slot]
+  // [item slot] K_j and V_j of the item; once the item's last products have
+  // read them, the same bytes stage its dK and dV tiles (bf16, 128-byte
+  // swizzle) on their way to global memory.
+  uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
   uint8_t q[kStages][kTileBytes];
   uint8_t dout[kStages][kTileBytes];
@@ -226,12 +229,35 @@ struct alignas(1024) Smem {
   uint64_t kv_full[2], kv_empty[2];
   uint64_t in_full[kStages], in_empty[kStages];
   uint64_t sdp_full, sdp_free, ds_full, pds_free;
+  uint64_t ostage_full;  // the finished item's dK/dV rows are staged
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
 };
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 static_assert(kSmemBytes <= 232448, "dK/dV shared memory exceeds the 227 KiB per-block limit");
+
+// Row r's 16 columns [16g, 16g + 16) of dV and of dK * scale, as bf16, into
+// the staging tiles (128-byte swizzle: 16-byte chunk c of row r at
+// r * 128 + ((c ^ (r & 7)) << 4)); chunks 2g and 2g + 1.
+__device__ __forceinline__ void stage_dkdv_row(uint8_t* dk_tile, uint8_t* dv_tile,
+                                               const uint32_t (&av)[16], const uint32_t (&ak)[16],
+                                               int r, int g, float s) {
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    const int off = r * 128 + (((2 * g + v) ^ (r & 7)) << 4);
+    *reinterpret_cast<uint4*>(dv_tile + off) =
+        make_uint4(pack_bf16(__uint_as_float(av[8 * v]), __uint_as_float(av[8 * v + 1])),
+                   pack_bf16(__uint_as_float(av[8 * v + 2]), __uint_as_float(av[8 * v + 3])),
+                   pack_bf16(__uint_as_float(av[8 * v + 4]), __uint_as_float(av[8 * v + 5])),
+                   pack_bf16(__uint_as_float(av[8 * v + 6]), __uint_as_float(av[8 * v + 7])));
+    *reinterpret_cast<uint4*>(dk_tile + off) =
+        make_uint4(pack_bf16(__uint_as_float(ak[8 * v]) * s, __uint_as_float(ak[8 * v + 1]) * s),
+                   pack_bf16(__uint_as_float(ak[8 * v + 2]) * s, __uint_as_float(ak[8 * v + 3]) * s),
+                   pack_bf16(__uint_as_float(ak[8 * v + 4]) * s, __uint_as_float(ak[8 * v + 5]) * s),
+                   pack_bf16(__uint_as_float(ak[8 * v + 6]) * s, __uint_as_float(ak[8 * v + 7]) * s));
+  }
+}
 
 __device__ __forceinline__ void decode(int k, const AttnShape& sh, int& b, int& h, int& j) {
   const int bh_count = sh.B * sh.H;
@@ -243,9 +269,9 @@ __device__ __forceinline__ void decode(int k, const AttnShape& sh, int& b, int& 
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
-                     const __grid_constant__ CUtensorMap map_do, const float* __restrict__ lse,
-                     const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv,
-                     const AttnShape sh) {
+                     const __grid_constant__ CUtensorMap map_do,
+                     const __grid_constant__ CUtensorMap map_dqkv, const float* __restrict__ lse,
+                     const float* __restrict__ delta, const AttnShape sh) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
@@ -259,7 +285,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+      // The item's last products (commit) and the store of its dK/dV tiles
+      // out of the same bytes (lane 0 of warp 0, once the bulk stores have
+      // read them).
+      mbar_init(&sm.kv_empty[s], 2);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.in_full[s], 2);  // TMA bytes + the warp's lse/Delta stores
@@ -269,6 +298,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
     mbar_init(&sm.sdp_free, kEwWarps);
     mbar_init(&sm.ds_full, kEwWarps);
     mbar_init(&sm.pds_free, 1);
+    mbar_init(&sm.ostage_full, kEwWarps);
     mbar_init(&sm.drain[0], 1);
     mbar_init(&sm.drain[1], 1);
     sm.abort = 0;
@@ -291,6 +321,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&map_qkv);
     tma_prefetch_desc(&map_do);
+    tma_prefetch_desc(&map_dqkv);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -468,7 +499,37 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
     const uint32_t t_p = tmem + lb + 256 + 16 * g, t_ds = tmem + lb + 320 + 16 * g;
     const uint32_t t_dv = tmem + lb + 384 + 16 * g, t_dk = tmem + lb + 448 + 16 * g;
     const float sc = sh.scale_log2;
-    uint32_t sdp_cnt = 0, pds_cnt = 0, in_it = 0;
+    uint32_t sdp_cnt = 0, pds_cnt = 0, in_it = 0, ost_cnt = 0;
+    // The finished item's dK and dV rows go to global memory through the
+    // item's own K and V tiles (slot `ps`), which its last products have
+    // finished reading (the item's last dV/dK product completed before this
+    // warp read the accumulators): every warp writes its rows there, and lane
+    // 0 of warp 0 stores both 128 x 64 tiles with two TMA bulk stores (dqkv
+    // slots 1 and 2; rows past T are clipped), then releases the slot to the
+    // loads of the item after next. Scattered 32-byte stores from every
+    // thread, one segment per row, held all 16 warps for ~2000 cycles per
+    // item. Returns false if a wait gave up.
+    auto emit_dkdv = [&](const uint32_t (&av)[16], const uint32_t (&ak)[16], int eb, int eh,
+                         int ej, int ps) -> bool {
+      stage_dkdv_row(sm.k[ps], sm.v[ps], av, ak, r, g, sh.scale);
+      fence_proxy_async_smem();  // generic-proxy writes, read by the TMA engine
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.ostage_full);
+      bool w = true;
+      if (warp == 0 && lane == 0) {
+        w = mbar_wait(&sm.ostage_full, ost_cnt & 1, kSiteDkvSoftmax, abort);
+        if (w) {
+          tma_store_3d(&map_dqkv, sm.k[ps], C + eh * kD, ej * kBlockN, eb);
+          tma_store_3d(&map_dqkv, sm.v[ps], 2 * C + eh * kD, ej * kBlockN, eb);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(&sm.kv_empty[ps]);
+        }
+      }
+      ++ost_cnt;
+      return __all_sync(0xffffffffu, w);
+    };
+    int item_cnt = 0, ps = 0;
     // The finished item whose dV, dK still sit in tensor memory: they are read
     // out while the next item's first tile is processed, just before its P^T
     // and dS^T go to tensor memory (after which the next dV/dK product
@@ -535,7 +596,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.ds_full);
-          store_dkdv_row(dqkv, av, ak, pb, ph, pj, r, g, C, sh);
+          ok = emit_dkdv(av, ak, pb, ph, pj, ps);
+          if (!ok) break;
           pending = false;
         } else {
           tmem_st16(t_p, pp);
@@ -551,6 +613,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
       pb = b;
       ph = h;
       pj = j;
+      ps = item_cnt & 1;
+      ++item_cnt;
     }
     if (ok && pending) {
       ok = mbar_wait(&sm.pds_free, pds_cnt & 1, kSiteDkvSoftmax, abort);
@@ -563,9 +627,12 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_qkv,
         tmem_ld16(t_dk, ak);
         tmem_wait_ld();
         tc_fence_before();
-        store_dkdv_row(dqkv, av, ak, pb, ph, pj, r, g, C, sh);
+        emit_dkdv(av, ak, pb, ph, pj, ps);
       }
     }
+    // Every bulk store this CTA issued has completed before it exits.
+    if (warp == 0 && lane == 0) bulk_wait_group0();
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -470,9 +470,11 @@ ga_status gpt2_attn_bwd_dkdv(const void* qkv, const void* dout, const float* lse
   BwdLaunch L;
   const ga_status st = prepare_bwd(qkv, dout, lse, delta, dqkv, B, T, H, D, scale, &L);
   if (st != GA_OK) return st;
+  CUtensorMap map_dqkv;
+  if (!make_map(&map_dqkv, dqkv, static_cast<uint64_t>(3) * H * kD, T, B)) return GA_ERR_CUDA;
   ga::bwd::dkdv::attn_bwd_dkdv_kernel<<<L.grid, ga::bwd::kThreads, ga::bwd::dkdv::kSmemBytes,
                                         reinterpret_cast<cudaStream_t>(stream)>>>(
-      L.map_qkv, L.map_do, lse, delta, static_cast<__nv_bfloat16*>(dqkv), L.sh);
+      L.map_qkv, L.map_do, map_dqkv, lse, delta, L.sh);
   return check_launch();
 }
 

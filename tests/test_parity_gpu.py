@@ -267,10 +267,12 @@ def test_fused_backward_full_size_and_deterministic(ops):
     (1, 1, 1, [0]),                      # a single token
     (2, 300, 3, [0, 1, 127, 128, 255, 256, 299]),   # chunk edges and the last row
     (1, 1000, 2, [511, 512, 999]),
+    (1, 2100, 2, [1023, 1024, 2099]),    # 8, 9 and 17 chunks
 ])
 def test_decode_matches_oracle_row(ops, B, T, H, ts):
     """Decode attention of row t equals row t of the causal forward: out and
-    lse against the oracle, at chunk boundaries and the last row."""
+    lse against the oracle, at chunk boundaries and the last row, and for rows
+    longer than the bench's T = 1024."""
     qkv_bf, _ = make_inputs(B, T, H, 64, seed=40 + T)
     qkv = qkv_bf.cuda()
     out_o, lse_o = orc.attention_forward(qkv_bf.double().numpy(), 0.125)
