@@ -14,16 +14,20 @@
 //   attn_decode_partial_kernel  one CTA (4 warps) per (chunk, h, b). One
 //       thread issues two TMA box loads at once, the chunk's 128 k rows and
 //       its 128 v rows (16 KiB each, the forward's packed-qkv tensor map,
-//       128-byte swizzle), so every byte the CTA needs is in flight from its
-//       first instruction; with 32 KiB of shared memory per CTA, seven CTAs
-//       per SM keep the whole grid's loads streaming. Thread r then scores
-//       key r against q (held in registers) from shared memory; the block
-//       takes its max and sum in base 2; and each warp accumulates p * v over
-//       its 32 keys, each lane owning two of the 64 columns. The four warps
-//       are combined and the chunk's (max, sum, unnormalised o) goes to the
+//       128-byte swizzle, each on its own mbarrier), so every byte the CTA
+//       needs is in flight from its first instruction and the scores start
+//       as soon as the k rows land. At 36 KiB of shared memory per CTA (with
+//       the alignment slack and the per-CTA reserve), six CTAs fit on an SM:
+//       888 resident CTAs hold 28 MiB of loads in flight. Thread r scores key
+//       r against q (held in registers) from shared memory; the block takes
+//       its max and sum in base 2; and each warp accumulates p * v over its 32
+//       keys, each lane owning two of the 64 columns. The four warps are
+//       combined and the chunk's (max, sum, unnormalised o) goes to the
 //       workspace.
 //   attn_decode_combine_kernel  one CTA per (h, b): merges the chunks
-//       (rescaling each by 2^(m_c - m)) into out (bf16) and the natural-log lse.
+//       (rescaling each by 2^(m_c - m)) into out (bf16) and the natural-log
+//       lse; a programmatic dependent launch, so its CTAs are resident and
+//       waiting when the partials land.
 #pragma once
 
 #include "common.cuh"
@@ -49,7 +53,7 @@ struct alignas(1024) Smem {
   float p[kChunk];
   float red[2][kWarps];
   float o[kWarps][kD];
-  uint64_t full;
+  uint64_t full_k, full_v;  // the chunk's k rows, v rows landed
   int abort;
 };
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
@@ -75,17 +79,22 @@ attn_decode_partial_kernel(const __grid_constant__ CUtensorMap map_qkv,
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
+  // The combine kernel may be scheduled now; it waits for this grid's
+  // writes before reading them.
+  grid_dependents_launch();
   const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = sh.H * kD;
   const int c0 = chunk * kChunk;
   if (threadIdx.x == 0) {
-    mbar_init(&sm.full, 1);
+    mbar_init(&sm.full_k, 1);
+    mbar_init(&sm.full_v, 1);
     sm.abort = 0;
     fence_barrier_init();
-    mbar_arrive_expect_tx(&sm.full, 2 * kTileBytes);
-    tma_load_3d(sm.k, &map_qkv, &sm.full, C + h * kD, c0, b);
-    tma_load_3d(sm.v, &map_qkv, &sm.full, 2 * C + h * kD, c0, b);
+    mbar_arrive_expect_tx(&sm.full_k, kTileBytes);
+    tma_load_3d(sm.k, &map_qkv, &sm.full_k, C + h * kD, c0, b);
+    mbar_arrive_expect_tx(&sm.full_v, kTileBytes);
+    tma_load_3d(sm.v, &map_qkv, &sm.full_v, 2 * C + h * kD, c0, b);
   }
   // q of row t (every thread reads the same 128 bytes), meanwhile.
   const size_t row_elems = static_cast<size_t>(3) * C;
@@ -100,7 +109,8 @@ attn_decode_partial_kernel(const __grid_constant__ CUtensorMap map_qkv,
     q[4 * c + 3] = w.w;
   }
   __syncthreads();  // the barrier is initialised before anyone waits on it
-  const bool ok = mbar_wait(&sm.full, 0, kSiteDecode, &sm.abort);
+  // The scores need only k; v is waited for before the p * v step.
+  bool ok = mbar_wait(&sm.full_k, 0, kSiteDecode, &sm.abort);
   // Every thread leaves through the same barriers below; a thread whose wait
   // gave up computes on whatever is in shared memory and nothing is written.
   const int key = c0 + threadIdx.x;
@@ -129,6 +139,7 @@ attn_decode_partial_kernel(const __grid_constant__ CUtensorMap map_qkv,
   const float l = warp_sum(p);
   if (lane == 0) sm.red[1][warp] = l;
   __syncthreads();
+  ok = mbar_wait(&sm.full_v, 0, kSiteDecode, &sm.abort) && ok;
   // o[2*lane .. 2*lane+1] = sum over this warp's 32 keys of p * v.
   float o0 = 0.f, o1 = 0.f;
   const int cpair = lane >> 2;         // 16-byte chunk holding columns 2*lane, 2*lane+1
@@ -147,7 +158,10 @@ attn_decode_partial_kernel(const __grid_constant__ CUtensorMap map_qkv,
   if (__syncthreads_or(!ok)) {
     // A wait gave up: nothing is written; the loads still in flight are
     // waited for (bounded) before the CTA's shared memory goes away.
-    if (threadIdx.x == 0) drain_wait(&sm.full, 0, kSiteDecode);
+    if (threadIdx.x == 0) {
+      drain_wait(&sm.full_k, 0, kSiteDecode);
+      drain_wait(&sm.full_v, 0, kSiteDecode);
+    }
   } else {
     float* out = partials + ((static_cast<size_t>(b) * sh.H + h) * gridDim.x + chunk) * kPartialFloats;
     if (threadIdx.x < kD)
@@ -160,22 +174,49 @@ attn_decode_partial_kernel(const __grid_constant__ CUtensorMap map_qkv,
   }
 }
 
-// One CTA of 64 threads (one per column) per (h, b).
+// One CTA of 64 threads (one per column) per (h, b). The chunks are read in
+// batches of 8 with independent loads (one round trip to L2 per batch, not
+// one per chunk) and merged against a running max: a batch raises the max
+// M to include its chunks, rescales the sums so far by 2^(M_old - M), and
+// adds its chunks (each rescaled by 2^(m_c - M)) in chunk order. Rows of at
+// most 8 chunks are one batch. Launched as a programmatic dependent of the
+// partial kernel: the CTAs may start while the partials are still being
+// written, and wait for them (griddepcontrol.wait) before the first read.
 __global__ void __launch_bounds__(kD)
 attn_decode_combine_kernel(const float* __restrict__ partials, int n_chunks,
                            __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
                            const AttnShape sh) {
+  grid_dependency_wait();
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const float* p = partials + (static_cast<size_t>(b) * sh.H + h) * n_chunks * kPartialFloats;
-  float M = -INFINITY;
-  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, p[c * kPartialFloats]);
-  float L = 0.f, o = 0.f;
-  for (int c = 0; c < n_chunks; ++c) {
-    const float mc = p[c * kPartialFloats];
-    if (mc == -INFINITY) continue;
-    const float w = exp2f(mc - M);
-    L = fmaf(p[c * kPartialFloats + 1], w, L);
-    o = fmaf(p[c * kPartialFloats + 2 + d], w, o);
+  constexpr int kBatch = 8;
+  float M = -INFINITY, L = 0.f, o = 0.f;
+  for (int c0 = 0; c0 < n_chunks; c0 += kBatch) {
+    float mc[kBatch], lc[kBatch], oc[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const bool in = c0 + i < n_chunks;
+      const float* pc = p + (c0 + i) * kPartialFloats;
+      mc[i] = in ? pc[0] : -INFINITY;
+      lc[i] = in ? pc[1] : 0.f;
+      oc[i] = in ? pc[2 + d] : 0.f;
+    }
+    float Mb = M;
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) Mb = fmaxf(Mb, mc[i]);
+    if (M != -INFINITY) {
+      const float w = exp2f(M - Mb);
+      L *= w;
+      o *= w;
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      if (mc[i] == -INFINITY) continue;
+      const float w = exp2f(mc[i] - Mb);
+      L = fmaf(lc[i], w, L);
+      o = fmaf(oc[i], w, o);
+    }
+    M = Mb;
   }
   out[(static_cast<size_t>(b) * sh.H + h) * kD + d] = __float2bfloat16_rn(o / L);
   if (d == 0) lse[static_cast<size_t>(b) * sh.H + h] = (M + log2f(L)) * 0.69314718055994531f;

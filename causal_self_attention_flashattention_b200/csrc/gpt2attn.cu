@@ -564,8 +564,22 @@ ga_status gpt2_attn_decode(const void* qkv, int t, void* out, float* lse, void* 
   ga::decode::attn_decode_partial_kernel<<<dim3(n_chunks, H, B), ga::decode::kWarps * 32,
                                            ga::decode::kSmemBytes, s>>>(
       map_qkv, static_cast<const __nv_bfloat16*>(qkv), t, partials, sh);
-  ga::decode::attn_decode_combine_kernel<<<dim3(H, B), ga::kD, 0, s>>>(
-      partials, n_chunks, static_cast<__nv_bfloat16*>(out), lse, sh);
+  // The combine is a programmatic dependent of the partial kernel: its
+  // launch overlaps the partials' tail, and it waits for them on the device.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(H, B);
+  cfg.blockDim = dim3(ga::kD);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // A refused launch leaves its error for check_launch to record.
+  (void)cudaLaunchKernelEx(&cfg, ga::decode::attn_decode_combine_kernel,
+                           static_cast<const float*>(partials), n_chunks,
+                           static_cast<__nv_bfloat16*>(out), lse, sh);
   return check_launch();
 }
 
