@@ -265,7 +265,7 @@ def test_fused_backward_full_size_and_deterministic(ops):
 
 @pytest.mark.parametrize("B,T,H,ts", [
     (1, 1, 1, [0]),                      # a single token
-    (2, 300, 3, [0, 1, 127, 128, 255, 256, 299]),   # chunk edges and the last row
+    (2, 300, 3, [0, 1, 63, 64, 127, 128, 255, 256, 299]),   # chunk edges and the last row
     (1, 1000, 2, [511, 512, 999]),
     (1, 2100, 2, [1023, 1024, 2099]),    # 8, 9 and 17 chunks
 ])
