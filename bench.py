@@ -31,6 +31,10 @@ figure, not this library's result.
 with the bf16 forward on the same inputs for reference. --linear times the
 dense layers around attention (c_attn, c_proj) at the workload's B, T, C.
 
+--v16 times the inference path with v in fp16 from c_attn: the forward that
+reads it (gpt2_attn_fwd_v16) next to the bf16 forward on the same values, and
+c_attn writing the fp16 v slot (gpt2_attn_qkv_proj_v16).
+
 --decode times decode attention instead (gpt2_attn_decode: the newest row
 t = T-1 of every (b, h) over the keys and values of rows 0..T-1), one GPU,
 and prints its own line: bytes of k and v read per second against the
@@ -686,6 +690,71 @@ def run_fp8(args, wl):
     return 0
 
 
+def run_v16(args, wl):
+    """The fp16-v forward (gpt2_attn_fwd_v16) on the workload's q, k, v with
+    the v slot stored as fp16, next to the bf16 forward (gpt2_attn_fwd) on the
+    same values, and c_attn writing that qkv (gpt2_attn_qkv_proj_v16): forward
+    TFLOPS (2*B*H*T^2*D) against the measured bf16 peak (the products run in
+    bf16 and fp16, which share the peak)."""
+    import torch
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from causal_self_attention_flashattention_b200 import build
+    build.build()
+    from causal_self_attention_flashattention_b200 import ops
+    from causal_self_attention_flashattention_b200.workload import (attention_flops, make_inputs,
+                                                                   make_linear_inputs)
+
+    B, T, H, D, scale = wl.B, wl.T, wl.H, wl.D, wl.scale
+    C = H * D
+    qkv_cpu, _ = make_inputs(B, T, H, D, seed=0, qk_std=wl.qk_std)
+    q16_cpu = qkv_cpu.clone()
+    q16_cpu[:, :, 2] = qkv_cpu[:, :, 2].to(torch.float16).view(torch.bfloat16)
+    sets = [dict(qkv=qkv_cpu.to(dev), q16=q16_cpu.to(dev),
+                 out=torch.empty(B, T, H, D, dtype=torch.bfloat16, device=dev),
+                 lse=torch.empty(B, H, T, dtype=torch.float32, device=dev))
+            for _ in range(args.sets)]
+    stream = torch.cuda.current_stream()
+    n = len(sets)
+    ms_v16 = _time_device(lambda i: ops.attn_fwd_v16(sets[i % n]["q16"], scale, out=sets[i % n]["out"],
+                                                     lse=sets[i % n]["lse"], stream=stream),
+                          args.steps, args.warmup, stream)
+    ms_bf16 = _time_device(lambda i: ops.attn_fwd(sets[i % n]["qkv"], scale, out=sets[i % n]["out"],
+                                                  lse=sets[i % n]["lse"], stream=stream),
+                           args.steps, args.warmup, stream)
+    x, w, b = make_linear_inputs(B, T, C, 3 * C, seed=0)
+    lin_sets = [dict(x=x.to(dev), w=w.to(dev), b=b.to(dev),
+                     qkv=torch.empty(B, T, 3, H, D, dtype=torch.bfloat16, device=dev))
+                for _ in range(args.sets)]
+    ms_proj = _time_device(lambda i: ops.qkv_proj(lin_sets[i % n]["x"], lin_sets[i % n]["w"],
+                                                  lin_sets[i % n]["b"], H, qkv=lin_sets[i % n]["qkv"],
+                                                  stream=stream, v_fp16=True),
+                           args.steps, args.warmup, stream)
+    st, word = ops.last_device_status()
+    if st != ops.GA_OK:
+        raise RuntimeError(f"device status: {ops.status_string(st)} ({word:#x})")
+    fwd_flops, _ = attention_flops(B, T, H, D)
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    tf = fwd_flops / (ms_v16 * 1e-3) / 1e12
+    line = {
+        "metric": "causal attention forward TFLOPS, v in fp16 from c_attn (gpt2_attn_fwd_v16)",
+        "value": tf, "unit": "TFLOPS", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_v16, "higher_is_better": True, "dtype": "bf16 q,k / fp16 v",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": B, "T": T, "H": H, "D": D,
+                   "l2": f"{n} rotating input sets"},
+        "roofline": {"kernel": "fwd_v16", "bound": "tensor", "achieved": tf, "peak": peak,
+                     "unit": "TFLOP/s", "frac": tf / peak,
+                     "peak_source": f"bf16_tflops of {peak_src}"},
+        "bf16_fwd_ms": ms_bf16, "qkv_proj_v16_ms": ms_proj,
+        "gpu_launches": args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_linear(args, wl):
     """The dense layers around attention (gpt2_attn_qkv_proj, gpt2_attn_out_proj)
     at the workload's B, T and width C = 64 H: TFLOPS against the measured bf16
@@ -798,6 +867,8 @@ def main(argv=None):
                    help="time the FP8 forward (and its quantisation pass) instead")
     p.add_argument("--linear", action="store_true",
                    help="time the dense layers around attention (c_attn, c_proj) instead")
+    p.add_argument("--v16", action="store_true",
+                   help="time the forward that reads v in fp16 from c_attn instead")
     p.add_argument("--context", action="store_true",
                    help="time torch SDPA on the same workload, for context")
     args = p.parse_args(argv)
@@ -816,6 +887,8 @@ def main(argv=None):
         return run_fp8(args, wl)
     if args.linear:
         return run_linear(args, wl)
+    if args.v16:
+        return run_v16(args, wl)
     return run_ours(args, wl)
 
 

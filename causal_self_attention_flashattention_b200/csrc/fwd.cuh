@@ -146,11 +146,15 @@ __device__ __forceinline__ void store_row(const uint32_t (&o)[64], int b, int h,
 // multipliers. S = Q K^T then multiplies e4m3 operands (kind::f8f6f4) and the
 // softmax scale absorbs dequant[0] * dequant[1]; V becomes fp16 holding
 // e4m3 * 2^-8 exactly, and O is multiplied by 2^8 * dequant[2] at the end.
-template <bool kFp8>
+// kV16: the v slot of qkv already holds fp16 (q and k stay bf16), as the
+// c_attn GEMM writes it when asked; the convert warp then only passes each V
+// tile on (kFp8 must be false).
+template <bool kFp8, bool kV16 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
                 const __grid_constant__ CUtensorMap map_v8, __nv_bfloat16* __restrict__ out,
                 float* __restrict__ lse, const AttnShape sh, const float* __restrict__ dequant) {
+  static_assert(!(kFp8 && kV16), "the FP8 forward widens its own e4m3 V");
   constexpr int kQK = kQKBytes<kFp8>;
   extern __shared__ uint8_t smem_raw[];
   Smem<kFp8>& sm = *reinterpret_cast<Smem<kFp8>*>(
@@ -365,7 +369,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
             *reinterpret_cast<uint4*>(row + (((2 * c) ^ (rr & 7)) << 4)) = lo;
             *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ (rr & 7)) << 4)) = hi;
           }
-        } else {
+        } else if (!kV16) {
           uint4* tile = reinterpret_cast<uint4*>(sm.v[s]);
           // Running max of |v| over the converted fp16 values: a bf16 beyond
           // fp16's range rounds to inf, so inf or NaN here flags the tile.

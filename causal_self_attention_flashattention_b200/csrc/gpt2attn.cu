@@ -105,6 +105,10 @@ const DeviceInfo* setup_device(int dev) {
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(ga::fwd::kSmemBytes<true>)) != cudaSuccess)
     return nullptr;
+  if (cudaFuncSetAttribute(ga::fwd::attn_fwd_kernel<false, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::fwd::kSmemBytes<false>)) != cudaSuccess)
+    return nullptr;
   // The forward kernel's setmaxnreg split (warpgroup budgets that add up to the
   // block's allocation) is only safe if it launches with the register count
   // the split was sized for.
@@ -113,6 +117,9 @@ const DeviceInfo* setup_device(int dev) {
       fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
     return nullptr;
   if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel<true>) != cudaSuccess ||
+      fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
+    return nullptr;
+  if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel<false, true>) != cudaSuccess ||
       fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
     return nullptr;
 
@@ -307,8 +314,12 @@ size_t delta_bytes(int B, int T, int H) {
 
 extern "C" {
 
-ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int D,
-                        float scale, gpt2attn_stream_t stream) {
+namespace {
+
+// The bf16 forward, with v read as bf16 (converted in the kernel) or, for
+// v16, as fp16 already.
+ga_status launch_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int D,
+                     float scale, gpt2attn_stream_t stream, bool v16) {
   if (qkv == nullptr || out == nullptr || lse == nullptr) return GA_ERR_INVALID_ARG;
   ga_status st = check_shape(B, T, H, D);
   if (st != GA_OK) return st;
@@ -317,15 +328,34 @@ ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse, int B, int T, in
   const DeviceInfo* info = device_info();
   if (info == nullptr) return GA_ERR_CUDA;
 
+  // One 16-bit map serves q, k and v: a TMA copy moves bytes, whatever the
+  // 16-bit type.
   CUtensorMap map_qkv;
   if (!make_map(&map_qkv, qkv, static_cast<uint64_t>(3) * H * kD, T, B)) return GA_ERR_CUDA;
   const ga::AttnShape sh = make_shape(B, T, H, scale);
   const int items = ga::fwd::num_items(sh);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  ga::fwd::attn_fwd_kernel<false><<<grid_for(items, info->num_sms), ga::fwd::kThreads,
-                                    ga::fwd::kSmemBytes<false>, s>>>(
-      map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr);
+  if (v16)
+    ga::fwd::attn_fwd_kernel<false, true><<<grid_for(items, info->num_sms), ga::fwd::kThreads,
+                                            ga::fwd::kSmemBytes<false>, s>>>(
+        map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr);
+  else
+    ga::fwd::attn_fwd_kernel<false><<<grid_for(items, info->num_sms), ga::fwd::kThreads,
+                                      ga::fwd::kSmemBytes<false>, s>>>(
+        map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr);
   return check_launch();
+}
+
+}  // namespace
+
+ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int D,
+                        float scale, gpt2attn_stream_t stream) {
+  return launch_fwd(qkv, out, lse, B, T, H, D, scale, stream, false);
+}
+
+ga_status gpt2_attn_fwd_v16(const void* qkv, void* out, float* lse, int B, int T, int H, int D,
+                            float scale, gpt2attn_stream_t stream) {
+  return launch_fwd(qkv, out, lse, B, T, H, D, scale, stream, true);
 }
 
 ga_status gpt2_attn_fp8_quantize(const void* qkv, void* qkv8, float* scales, int B, int T, int H,
@@ -588,7 +618,7 @@ namespace {
 // y (M, N) = a (M, K) w (N, K)^T + bias (N): the shared body of the two dense
 // layers. K and N are multiples of 64 here (C = H * 64).
 ga_status launch_linear(const void* a, const void* w, const void* bias, void* y, long long M,
-                        int N, int K, gpt2attn_stream_t stream) {
+                        int N, int K, int f16_from, gpt2attn_stream_t stream) {
   if (static_cast<long double>(M) * (N > K ? N : K) >= 2147483648.0L) return GA_ERR_INVALID_ARG;
   const DeviceInfo* info = device_info();
   if (info == nullptr) return GA_ERR_CUDA;
@@ -604,7 +634,7 @@ ga_status launch_linear(const void* a, const void* w, const void* bias, void* y,
   g.N = N;
   g.K = K;
   g.tiles_n = ga::ceil_div(N, ga::linear::kBN);
-  g.f16_from = N;
+  g.f16_from = f16_from;
   const int tiles = ga::ceil_div(g.M, ga::linear::kBM) * g.tiles_n;
   ga::linear::linear_kernel<<<grid_for(tiles, info->num_sms), ga::linear::kThreads,
                               ga::linear::kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(
@@ -628,7 +658,19 @@ ga_status gpt2_attn_qkv_proj(const void* x, const void* w_attn, const void* b_at
   const ga_status st = check_linear_args(x, w_attn, b_attn, qkv, B, T, H, D);
   if (st != GA_OK) return st;
   const int C = H * D;
-  return launch_linear(x, w_attn, b_attn, qkv, static_cast<long long>(B) * T, 3 * C, C, stream);
+  return launch_linear(x, w_attn, b_attn, qkv, static_cast<long long>(B) * T, 3 * C, C, 3 * C,
+                       stream);
+}
+
+ga_status gpt2_attn_qkv_proj_v16(const void* x, const void* w_attn, const void* b_attn,
+                                 void* qkv, int B, int T, int H, int D,
+                                 gpt2attn_stream_t stream) {
+  const ga_status st = check_linear_args(x, w_attn, b_attn, qkv, B, T, H, D);
+  if (st != GA_OK) return st;
+  const int C = H * D;
+  // Columns [2C, 3C) are the v slot.
+  return launch_linear(x, w_attn, b_attn, qkv, static_cast<long long>(B) * T, 3 * C, C, 2 * C,
+                       stream);
 }
 
 ga_status gpt2_attn_out_proj(const void* out, const void* w_proj, const void* b_proj, void* y,
@@ -636,7 +678,7 @@ ga_status gpt2_attn_out_proj(const void* out, const void* w_proj, const void* b_
   const ga_status st = check_linear_args(out, w_proj, b_proj, y, B, T, H, D);
   if (st != GA_OK) return st;
   const int C = H * D;
-  return launch_linear(out, w_proj, b_proj, y, static_cast<long long>(B) * T, C, C, stream);
+  return launch_linear(out, w_proj, b_proj, y, static_cast<long long>(B) * T, C, C, C, stream);
 }
 
 ga_status gpt2_attn_selftest_wait_timeout(unsigned long long limit_ns, gpt2attn_stream_t stream) {

@@ -50,6 +50,8 @@ EXPORTED_SYMBOLS = (
     "gpt2_attn_last_device_status",
     "gpt2_attn_selftest_wait_timeout",
     "gpt2_attn_qkv_proj",
+    "gpt2_attn_qkv_proj_v16",
+    "gpt2_attn_fwd_v16",
     "gpt2_attn_fp8_quantize",
     "gpt2_attn_fwd_fp8",
     "gpt2_attn_out_proj",
@@ -98,6 +100,10 @@ _lib.gpt2_attn_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
 _lib.gpt2_attn_fwd_fp8.restype = _i
 _lib.gpt2_attn_qkv_proj.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
 _lib.gpt2_attn_qkv_proj.restype = _i
+_lib.gpt2_attn_qkv_proj_v16.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+_lib.gpt2_attn_qkv_proj_v16.restype = _i
+_lib.gpt2_attn_fwd_v16.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+_lib.gpt2_attn_fwd_v16.restype = _i
 _lib.gpt2_attn_out_proj.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
 _lib.gpt2_attn_out_proj.restype = _i
 _lib.gpt2_attn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, _vp]
@@ -168,8 +174,15 @@ def default_scale(D: int) -> float:
 
 
 def attn_fwd(qkv: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None,
-             lse: torch.Tensor | None = None, stream=None):
-    """Causal attention forward: returns (out (B,T,H,D) bf16, lse (B,H,T) fp32)."""
+             lse: torch.Tensor | None = None, stream=None, check_status: bool = False):
+    """Causal attention forward: returns (out (B,T,H,D) bf16, lse (B,H,T) fp32).
+
+    The P V product runs in fp16, so every v entry must lie within fp16's
+    range (|v| <= 65504, finite). An entry outside it is reported on the
+    device as GA_ERR_RANGE, and out is then undefined. The call itself is
+    asynchronous and does not see that report; with check_status=True it
+    synchronises the stream afterwards and raises AttnError on any device
+    report (GA_ERR_RANGE, or GA_ERR_TIMEOUT from a wait that gave up)."""
     B, T, H, D = _dims(qkv)
     _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
     scale = default_scale(D) if scale is None else float(scale)
@@ -181,6 +194,29 @@ def attn_fwd(qkv: torch.Tensor, scale: float | None = None, out: torch.Tensor | 
     _expect(lse, "lse", (B, H, T), torch.float32)
     _check(_lib.gpt2_attn_fwd(qkv.data_ptr(), out.data_ptr(), lse.data_ptr(), B, T, H, D,
                               scale, _stream_ptr(stream)), "gpt2_attn_fwd")
+    if check_status:
+        st, word = last_device_status(stream)
+        if st != GA_OK:
+            raise AttnError(st, f"gpt2_attn_fwd (device report {word:#x})")
+    return out, lse
+
+
+def attn_fwd_v16(qkv: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None,
+                 lse: torch.Tensor | None = None, stream=None):
+    """attn_fwd for a qkv whose v slot holds fp16 bits (q, k bf16), as
+    qkv_proj(..., v_fp16=True) writes it: returns (out, lse) without the
+    kernel's bf16 -> fp16 conversion of V. Inference and prefill only."""
+    B, T, H, D = _dims(qkv)
+    _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
+    scale = default_scale(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=qkv.device)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=qkv.device)
+    _expect(out, "out", (B, T, H, D), torch.bfloat16)
+    _expect(lse, "lse", (B, H, T), torch.float32)
+    _check(_lib.gpt2_attn_fwd_v16(qkv.data_ptr(), out.data_ptr(), lse.data_ptr(), B, T, H, D,
+                                  scale, _stream_ptr(stream)), "gpt2_attn_fwd_v16")
     return out, lse
 
 
@@ -382,11 +418,12 @@ def last_device_status(stream=None) -> tuple[int, int]:
 
 
 class CausalSelfAttention(torch.autograd.Function):
-    """Autograd wrapper: y = attention(qkv), with both passes in the library."""
+    """Autograd wrapper: y = attention(qkv), with both passes in the library.
+    The forward's fp16 limit on v applies (see attn_fwd)."""
 
     @staticmethod
-    def forward(ctx, qkv, scale=None):
-        out, lse = attn_fwd(qkv, scale)
+    def forward(ctx, qkv, scale=None, check_status=False):
+        out, lse = attn_fwd(qkv, scale, check_status=check_status)
         ctx.save_for_backward(qkv, out, lse)
         ctx.scale = scale
         return out
@@ -394,19 +431,28 @@ class CausalSelfAttention(torch.autograd.Function):
     @staticmethod
     def backward(ctx, dout):
         qkv, out, lse = ctx.saved_tensors
-        return attn_bwd(qkv, out, dout.contiguous(), lse, ctx.scale), None
+        return attn_bwd(qkv, out, dout.contiguous(), lse, ctx.scale), None, None
 
 
-def causal_self_attention(qkv: torch.Tensor, scale: float | None = None) -> torch.Tensor:
-    """One-call causal self-attention on packed qkv (B,T,3,H,D) -> (B,T,H,D)."""
-    return CausalSelfAttention.apply(qkv, scale)
+def causal_self_attention(qkv: torch.Tensor, scale: float | None = None,
+                          check_status: bool = False) -> torch.Tensor:
+    """One-call causal self-attention on packed qkv (B,T,3,H,D) -> (B,T,H,D).
+
+    Every v entry must lie within fp16's range (|v| <= 65504): the forward's
+    P V product runs in fp16. check_status=True synchronises after the
+    forward and raises AttnError if the device reported a v entry outside it
+    (or a wait that gave up); otherwise out is undefined in that case."""
+    return CausalSelfAttention.apply(qkv, scale, check_status)
 
 
 def qkv_proj(x: torch.Tensor, w_attn: torch.Tensor, b_attn: torch.Tensor, H: int,
-             qkv: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+             qkv: torch.Tensor | None = None, stream=None, v_fp16: bool = False) -> torch.Tensor:
     """c_attn: qkv = x W_attn^T + b_attn, returned as packed (B, T, 3, H, D) bf16.
 
     x (B, T, C) bf16, w_attn (3C, C) bf16 (nn.Linear layout), b_attn (3C,) bf16.
+    With v_fp16=True the v slot holds fp16 bits (read it as
+    qkv[:, :, 2].view(torch.float16)): the input of attn_fwd_v16, not of
+    attn_fwd or attn_bwd.
     """
     if x.dim() != 3:
         raise ValueError(f"x must be (B, T, C), got {tuple(x.shape)}")
@@ -420,9 +466,10 @@ def qkv_proj(x: torch.Tensor, w_attn: torch.Tensor, b_attn: torch.Tensor, H: int
     if qkv is None:
         qkv = torch.empty((B, T, 3, H, D), dtype=torch.bfloat16, device=x.device)
     _expect(qkv, "qkv", (B, T, 3, H, D), torch.bfloat16)
-    _check(_lib.gpt2_attn_qkv_proj(x.data_ptr(), w_attn.data_ptr(), b_attn.data_ptr(),
-                                   qkv.data_ptr(), B, T, H, D, _stream_ptr(stream)),
-           "gpt2_attn_qkv_proj")
+    fn = _lib.gpt2_attn_qkv_proj_v16 if v_fp16 else _lib.gpt2_attn_qkv_proj
+    _check(fn(x.data_ptr(), w_attn.data_ptr(), b_attn.data_ptr(), qkv.data_ptr(), B, T, H, D,
+              _stream_ptr(stream)),
+           "gpt2_attn_qkv_proj_v16" if v_fp16 else "gpt2_attn_qkv_proj")
     return qkv
 
 

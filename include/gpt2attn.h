@@ -85,6 +85,19 @@ ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse,
                         gpt2attn_stream_t stream);
 
 /*
+ * gpt2_attn_fwd for a qkv whose v slot already holds fp16 (q and k bf16), as
+ * gpt2_attn_qkv_proj_v16 writes it: the same computation and outputs, without
+ * the in-kernel bf16 -> fp16 conversion of each V tile (the P V product runs
+ * in fp16 either way). For a v that bf16 and fp16 both hold exactly, out and
+ * lse are bit-identical to gpt2_attn_fwd's on the bf16 qkv. For inference
+ * and prefill: the backward reads v as bf16. Same arguments, layout and
+ * errors as gpt2_attn_fwd, except that no v range check is needed (no
+ * GA_ERR_RANGE).
+ */
+ga_status gpt2_attn_fwd_v16(const void* qkv, void* out, float* lse, int B, int T, int H, int D,
+                            float scale, gpt2attn_stream_t stream);
+
+/*
  * Size in bytes of the workspace gpt2_attn_bwd needs for this shape:
  * Delta, fp32 (B,H,T), at offset 0, rounded up to 256 bytes, where
  * Delta[b,h,t] = sum_d dout[b,t,h,d] * out[b,t,h,d]. After a gpt2_attn_bwd
@@ -281,6 +294,15 @@ ga_status gpt2_attn_fwd_fp8(const void* qkv8, const float* scales, void* out, fl
 ga_status gpt2_attn_qkv_proj(const void* x, const void* w_attn, const void* b_attn,
                              void* qkv, int B, int T, int H, int D,
                              gpt2attn_stream_t stream);
+/*
+ * As gpt2_attn_qkv_proj, but the v slot of qkv (columns [2C, 3C)) is written
+ * in fp16 (round to nearest; |v| above 65504 becomes inf), q and k in bf16:
+ * the input gpt2_attn_fwd_v16 reads. A qkv written this way is not an input
+ * of gpt2_attn_fwd or of the backward, which read v as bf16.
+ */
+ga_status gpt2_attn_qkv_proj_v16(const void* x, const void* w_attn, const void* b_attn,
+                                 void* qkv, int B, int T, int H, int D,
+                                 gpt2attn_stream_t stream);
 ga_status gpt2_attn_out_proj(const void* out, const void* w_proj, const void* b_proj,
                              void* y, int B, int T, int H, int D,
                              gpt2attn_stream_t stream);

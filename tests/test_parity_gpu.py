@@ -459,6 +459,17 @@ def test_v_outside_fp16_range_is_reported(ops, v_val, flagged):
         assert st == ops.GA_OK and word == 0, (st, hex(word))
         assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
     assert ops.last_device_status() == (ops.GA_OK, 0)
+    # The same report through the binding's opt-in check, and the autograd
+    # wrapper's.
+    if flagged:
+        with pytest.raises(ops.AttnError):
+            ops.attn_fwd(qkv, check_status=True)
+        with pytest.raises(ops.AttnError):
+            ops.causal_self_attention(qkv, check_status=True)
+    else:
+        ops.attn_fwd(qkv, check_status=True)
+        ops.causal_self_attention(qkv, check_status=True)
+    assert ops.last_device_status() == (ops.GA_OK, 0)
 
 
 def test_status_word_clean_after_runs(ops):
