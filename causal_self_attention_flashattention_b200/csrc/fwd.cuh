@@ -64,7 +64,7 @@ static_assert(kProducerWarp == 8 && kConvertWarp == 11, "warps 8-11 form the aux
 // powers of two; until then P may reach 2^8 (well inside fp16).
 constexpr float kRescaleLog2 = 8.f;
 // One pair in kPolyEvery is exponentiated with the FMA-pipe polynomial.
-constexpr int kPolyEvery = 4;
+constexpr int kPolyEvery = 6;
 constexpr uint32_t kTmemCols = 512;
 
 __device__ __forceinline__ uint32_t col_s(int q) { return q * 128; }

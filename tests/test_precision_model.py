@@ -4,7 +4,7 @@ forward kernel's arithmetic, checked against the oracle on CPU.
 The model follows the kernel step by step for one head: S = Q K^T in fp32
 from bf16 inputs; per 128-key tile, the row max with the stale-max rule
 (raised only when it grows by more than 2^8 in base 2), p = 2^(s*c - m*c)
-with every 4th pair of columns on the FMA-pipe polynomial, the row sum in the
+with every 6th pair of columns on the FMA-pipe polynomial, the row sum in the
 kernel's order, P packed to fp16 (round half up) and multiplied with V
 converted to fp16 (the integer conversion: exact down to 2^-14), O rescaled when the max is raised; at the end
 out = bf16(O / l) and lse = ln2 * (m*c + log2 l). Replacing the fp16 P and V
@@ -22,7 +22,9 @@ from .test_kernel_arith import (_bf16_rne, bf16x2_to_f16x2_model, exp2_poly_mode
 from .test_parity_gpu import LSE_TOL, out_error_ok
 
 LOG2E = 1.4426950408889634
-POLY_COLS = np.array([(col // 2) % 4 == 3 for col in range(128)])
+# The forward's kPolyEvery: pair c2 = col // 2 uses the polynomial when
+# c2 % 6 == 5.
+POLY_COLS = np.array([(col // 2) % 6 == 5 for col in range(128)])
 
 
 def v_to_f16_model(V):
