@@ -57,6 +57,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
+  int pair_clusters = 0;  // CTA pairs of the pair GEMM resident at once
 };
 
 std::mutex g_mutex;
@@ -131,9 +132,30 @@ const DeviceInfo* setup_device(int dev) {
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(ga::bwd::fused::kSmemBytes)) != cudaSuccess)
     return nullptr;
-  if (cudaFuncSetAttribute(ga::linear::linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(ga::linear::kSmemBytes)) != cudaSuccess)
+  if (cudaFuncSetAttribute(ga::linear::linear_pair_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::linear::kPairSmemBytes)) != cudaSuccess)
     return nullptr;
+  {
+    // How many two-CTA clusters fit at once (a pair must share a GPC, so an
+    // odd SM count in a GPC leaves one SM out).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (info.num_sms / 2));
+    cfg.blockDim = dim3(ga::linear::kThreads);
+    cfg.dynamicSmemBytes = ga::linear::kPairSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, ga::linear::linear_pair_kernel, &cfg) != cudaSuccess ||
+        n < 1)
+      return nullptr;
+    info.pair_clusters = n;
+  }
   if (cudaFuncSetAttribute(ga::bwd::dq::attn_bwd_dq_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(ga::bwd::dq::kSmemBytes)) != cudaSuccess)
@@ -623,22 +645,33 @@ ga_status launch_linear(const void* a, const void* w, const void* bias, void* y,
   const DeviceInfo* info = device_info();
   if (info == nullptr) return GA_ERR_CUDA;
   CUtensorMap map_a, map_w;
-  if (!make_map_2d(&map_a, a, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                   ga::linear::kBM))
+  if (!make_map_2d(&map_a, a, static_cast<uint64_t>(K), static_cast<uint64_t>(M), 128))
     return GA_ERR_CUDA;
-  if (!make_map_2d(&map_w, w, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
-                   ga::linear::kBN))
+  if (!make_map_2d(&map_w, w, static_cast<uint64_t>(K), static_cast<uint64_t>(N), 128))
     return GA_ERR_CUDA;
   ga::linear::GemmShape g;
   g.M = static_cast<int>(M);
   g.N = N;
   g.K = K;
-  g.tiles_n = ga::ceil_div(N, ga::linear::kBN);
   g.f16_from = f16_from;
-  const int tiles = ga::ceil_div(g.M, ga::linear::kBM) * g.tiles_n;
-  ga::linear::linear_kernel<<<grid_for(tiles, info->num_sms), ga::linear::kThreads,
-                              ga::linear::kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(
-      map_a, map_w, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(y), g);
+  // CTA pairs, each on 256 x 256 tiles of y.
+  const int tiles = ga::linear::num_pair_tiles(g);
+  const int clusters = tiles < info->pair_clusters ? tiles : info->pair_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(ga::linear::kThreads);
+  cfg.dynamicSmemBytes = ga::linear::kPairSmemBytes;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // A refused launch leaves its error for check_launch to record.
+  (void)cudaLaunchKernelEx(&cfg, ga::linear::linear_pair_kernel, map_a, map_w,
+                           static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(y), g);
   return check_launch();
 }
 

@@ -10,19 +10,11 @@
 // a layout pass: both are this one GEMM, y = A W^T + bias, written straight
 // into the layout the next step reads.
 //
-// sm_100a design: a persistent CTA per SM walks 128 x 256 output tiles.
-//   * Warp 0 (TMA): streams 128 x 64 tiles of A and 256 x 64 tiles of W
-//     (128-byte swizzle, rows past M or N read as zero) through a 4-stage
-//     ring.
-//   * Warp 1 (MMA, one thread): four tcgen05.mma M128 N256 K16 per stage into
-//     one of two 256-column fp32 accumulators in tensor memory, so the next
-//     tile's products run while the previous tile's epilogue reads out.
-//   * Warps 2-5 (epilogue): each thread owns one output row (its TMEM lane),
-//     adds the bias (read as one broadcast load per 8 columns), rounds to bf16
-//     (or fp16 for columns at or beyond `f16_from`) and stores 16-byte pieces
-//     of its row. No barrier other than the bounded mbarrier waits joins the
-//     epilogue warps, so a wait that gives up cannot strand the others.
-// Every wait is bounded like the attention kernels'.
+// sm_100a design: persistent two-CTA clusters (SM pairs) walk 256 x 256
+// output tiles; the pair's tensor-core products (tcgen05 .cta_group::2)
+// read half of each operand tile from each SM, so an SM loads 32 KiB of
+// operands per K step of 64 instead of the 48 KiB a one-SM 128 x 256 tile
+// needs. Every wait is bounded like the attention kernels'.
 #pragma once
 
 #include "common.cuh"
@@ -31,109 +23,142 @@
 namespace ga {
 namespace linear {
 
-constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kStages = 4;
+constexpr int kBK = 64;
 constexpr int kThreads = 192;
 constexpr int kProducerWarp = 0, kMmaWarp = 1, kEpiWarp0 = 2;
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
-constexpr uint32_t kABytes = kBM * kBK * 2, kBBytes = kBN * kBK * 2;
 
-struct alignas(1024) Smem {
-  uint8_t a[kStages][kABytes];
-  uint8_t b[kStages][kBBytes];
-  uint64_t full[kStages], empty[kStages];
+struct GemmShape {
+  int M, N, K;
+  int f16_from;  // columns >= f16_from are written as fp16 (N: none)
+};
+
+// ---------------------------------------------------------------------------
+// A two-CTA cluster computes a 256 x 256 tile of y: CTA r loads rows
+// [128 r, 128 r + 128) of the tile's A rows and the same half of its W rows;
+// one thread of CTA 0 issues tcgen05.mma .cta_group::2 M256 N256 K16, which
+// reads both CTAs' halves and leaves each CTA's 128 rows of the tile (all 256
+// columns) in that CTA's tensor memory.
+//   * Warp 0 of each CTA (TMA): its A and W halves into a 6-stage ring; the
+//     copies of both CTAs complete on CTA 0's `full` barrier (CTA 0 sets the
+//     stage's expected bytes for the pair).
+//   * Warp 1 of CTA 0 (MMA): waits on `full`, issues the pair's products and
+//     commits to `empty` in both CTAs; after a tile's last K step, to
+//     `acc_full` in both. Before a tile, it waits on CTA 0's `acc_empty`,
+//     which counts the eight epilogue warps of the pair.
+//   * Warps 2-5 of each CTA (epilogue): each thread owns one of the CTA's 128
+//     rows (its TMEM lane). It reads 128 accumulator columns per tensor-memory
+//     wait (32 columns per wait left the epilogue slower than the products),
+//     adds the bias (one broadcast load per 8 columns), rounds to bf16 (or
+//     fp16 for columns at or beyond `f16_from`) and stores 16-byte pieces of
+//     its row; then it arrives (remotely, from CTA 1) on CTA 0's `acc_empty`.
+//     No barrier other than the bounded mbarrier waits joins the epilogue
+//     warps, so a wait that gives up cannot strand the others.
+constexpr int kPairBM = 256, kPairBN = 256;
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairHalfBytes = 128 * kBK * 2;  // 16 KiB: a half tile of A or of W
+
+struct alignas(1024) PairSmem {
+  uint8_t a[kPairStages][kPairHalfBytes];
+  uint8_t b[kPairStages][kPairHalfBytes];
+  uint64_t full[kPairStages], empty[kPairStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
-static_assert(kSmemBytes <= 232448, "linear shared memory exceeds the 227 KiB per-block limit");
+constexpr size_t kPairSmemBytes = sizeof(PairSmem) + 1024;
+static_assert(kPairSmemBytes <= 232448, "pair GEMM shared memory exceeds the 227 KiB per-block limit");
 
-struct GemmShape {
-  int M, N, K;
-  int tiles_n;   // ceil(N / kBN)
-  int f16_from;  // columns >= f16_from are written as fp16 (N: none)
-};
-
-__device__ __forceinline__ int num_tiles(const GemmShape& g) {
-  return ceil_div(g.M, kBM) * g.tiles_n;
+__host__ __device__ __forceinline__ int num_pair_tiles(const GemmShape& g) {
+  return ceil_div(g.M, kPairBM) * ceil_div(g.N, kPairBN);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-linear_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
-              const uint16_t* __restrict__ bias, uint16_t* __restrict__ y,
-              const GemmShape g) {
+linear_pair_kernel(const __grid_constant__ CUtensorMap map_a,
+                   const __grid_constant__ CUtensorMap map_w, const uint16_t* __restrict__ bias,
+                   uint16_t* __restrict__ y, const GemmShape g) {
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                      ~uintptr_t(1023));
+  PairSmem& sm = *reinterpret_cast<PairSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_tiles = num_tiles(g);
+  const uint32_t rank = cluster_ctarank();
+  const int n_clusters = static_cast<int>(gridDim.x) / 2;
+  const int cid = static_cast<int>(blockIdx.x) / 2;
+  const int n_tiles = num_pair_tiles(g);
+  const int tiles_n = ceil_div(g.N, kPairBN);
   const int n_k = ceil_div(g.K, kBK);
   volatile int* abort = &sm.abort;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&sm.full[s], 1);   // used in CTA 0: its expect-tx arrival + both CTAs' bytes
+      mbar_init(&sm.empty[s], 1);  // the pair's commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.acc_full[b], 1);
-      mbar_init(&sm.acc_empty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&sm.acc_empty[b], 8);  // used in CTA 0: the pair's eight epilogue warps
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_barrier_init();
   }
-  if (warp == kProducerWarp && lane == 0) {
-    tma_prefetch_desc(&map_a);
-    tma_prefetch_desc(&map_w);
-  }
   if (warp == kMmaWarp) {
-    tmem_alloc(&sm.tmem_base, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(&sm.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialised and their tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  const uint32_t full0 = cluster_addr(&sm.full[0], 0);          // CTA 0's full[0]
+  const uint32_t acc_empty0 = cluster_addr(&sm.acc_empty[0], 0);  // CTA 0's acc_empty[0]
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
+      tma_prefetch_desc(&map_a);
+      tma_prefetch_desc(&map_w);
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-        const int tm = t / g.tiles_n, tn = t % g.tiles_n;
+      for (int t = cid; ok && t < n_tiles; t += n_clusters) {
+        const int tm = t / tiles_n, tn = t % tiles_n;
+        const int a_row = tm * kPairBM + static_cast<int>(rank) * 128;
+        const int w_row = tn * kPairBN + static_cast<int>(rank) * 128;
         for (int ks = 0; ks < n_k; ++ks, ++it) {
-          const int s = it % kStages;
-          if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, kSiteLinearProducer, abort)) {
+          const int s = it % kPairStages;
+          if (!mbar_wait(&sm.empty[s], ((it / kPairStages) & 1) ^ 1, kSiteLinearProducer, abort)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&sm.full[s], kABytes + kBBytes);
-          tma_load_2d(sm.a[s], &map_a, &sm.full[s], ks * kBK, tm * kBM);
-          tma_load_2d(sm.b[s], &map_w, &sm.full[s], ks * kBK, tn * kBN);
+          if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 4 * kPairHalfBytes);
+          tma_load_2d_pair(sm.a[s], &map_a, full0 + 8u * s, ks * kBK, a_row);
+          tma_load_2d_pair(sm.b[s], &map_w, full0 + 8u * s, ks * kBK, w_row);
         }
       }
-      for (int s = 0; s < kStages; ++s)
-        if (it > static_cast<uint32_t>(s))
-          drain_wait(&sm.full[s], ((it - s + kStages - 1) / kStages - 1) & 1, kSiteLinearProducer);
+      // CTA 0's full barriers count both CTAs' copies: waiting (bounded) for
+      // the last phase of each means no copy of either CTA is still landing
+      // (CTA 1 is held at the final cluster barrier until then).
+      if (rank == 0)
+        for (int s = 0; s < kPairStages; ++s)
+          if (it > static_cast<uint32_t>(s))
+            drain_wait(&sm.full[s], ((it - s + kPairStages - 1) / kPairStages - 1) & 1,
+                       kSiteLinearProducer);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kPairBM, kPairBN, 0, 0);
       uint32_t it = 0, lt = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++lt) {
+      for (int t = cid; ok && t < n_tiles; t += n_clusters, ++lt) {
         const uint32_t buf = lt & 1;
         if (!mbar_wait(&sm.acc_empty[buf], ((lt >> 1) & 1) ^ 1, kSiteLinearMma, abort)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + buf * kBN;
+        const uint32_t acc = tmem + buf * kPairBN;
         for (int ks = 0; ks < n_k; ++ks, ++it) {
-          const int s = it % kStages;
-          if (!mbar_wait(&sm.full[s], (it / kStages) & 1, kSiteLinearMma, abort)) {
+          const int s = it % kPairStages;
+          if (!mbar_wait(&sm.full[s], (it / kPairStages) & 1, kSiteLinearMma, abort)) {
             ok = false;
             break;
           }
@@ -142,39 +167,44 @@ linear_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.b[s]), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_ss(acc, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) ? 1u : 0u);
-          mma_commit(&sm.empty[s]);
+            mma_ss_pair(acc, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) ? 1u : 0u);
+          mma_commit_pair(&sm.empty[s]);
         }
         if (!ok) break;
-        mma_commit(&sm.acc_full[buf]);
+        mma_commit_pair(&sm.acc_full[buf]);
       }
-      mma_commit(&sm.drain);
+      // Every product has finished before either CTA frees its tensor memory.
+      mma_commit_pair(&sm.drain);
       drain_wait(&sm.drain, 0, kSiteLinearMma);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
-    const int r = q * 32 + lane;            // row within the tile
+    const int r = q * 32 + lane;            // row within this CTA's half of the tile
     uint32_t lt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++lt) {
-      const int tm = t / g.tiles_n, tn = t % g.tiles_n;
+    for (int t = cid; ok && t < n_tiles; t += n_clusters, ++lt) {
+      const int tm = t / tiles_n, tn = t % tiles_n;
       const uint32_t buf = lt & 1;
-      const int n0 = tn * kBN;
+      const int n0 = tn * kPairBN;
       ok = mbar_wait(&sm.acc_full[buf], (lt >> 1) & 1, kSiteLinearEpilogue, abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int row = tm * kBM + r;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kBN;
+      const int row = tm * kPairBM + static_cast<int>(rank) * 128 + r;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kPairBN;
       uint16_t* yrow = y + static_cast<size_t>(row) * g.N;
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(taddr + 32 * c, v);
+      for (int c4 = 0; c4 < kPairBN / 128; ++c4) {
+        uint32_t vv[4][32];
+#pragma unroll
+        for (int c1 = 0; c1 < 4; ++c1) tmem_ld32(taddr + 128 * c4 + 32 * c1, vv[c1]);
         tmem_wait_ld();
-        const int col0 = n0 + 32 * c;
+#pragma unroll
+        for (int c1 = 0; c1 < 4; ++c1) {
+        const uint32_t (&v)[32] = vv[c1];
+        const int col0 = n0 + 128 * c4 + 32 * c1;
         if (row < g.M) {
           const bool f16 = col0 >= g.f16_from;
 #pragma unroll
@@ -195,17 +225,18 @@ linear_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
             }
           }
         }
+        }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+      if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * buf);
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // no product, copy or tensor-memory read of either CTA outstanding
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
 }  // namespace linear
