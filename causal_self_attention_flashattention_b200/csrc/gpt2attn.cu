@@ -649,6 +649,9 @@ ga_status launch_linear(const void* a, const void* w, const void* bias, void* y,
     return GA_ERR_CUDA;
   if (!make_map_2d(&map_w, w, static_cast<uint64_t>(K), static_cast<uint64_t>(N), 128))
     return GA_ERR_CUDA;
+  CUtensorMap map_y;  // 16-bit y (bf16 or fp16 columns): the store only moves bits
+  if (!make_map_2d(&map_y, y, static_cast<uint64_t>(N), static_cast<uint64_t>(M), 32))
+    return GA_ERR_CUDA;
   ga::linear::GemmShape g;
   g.M = static_cast<int>(M);
   g.N = N;
@@ -670,8 +673,8 @@ ga_status launch_linear(const void* a, const void* w, const void* bias, void* y,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // A refused launch leaves its error for check_launch to record.
-  (void)cudaLaunchKernelEx(&cfg, ga::linear::linear_pair_kernel, map_a, map_w,
-                           static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(y), g);
+  (void)cudaLaunchKernelEx(&cfg, ga::linear::linear_pair_kernel, map_a, map_w, map_y,
+                           static_cast<const uint16_t*>(bias), g);
   return check_launch();
 }
 

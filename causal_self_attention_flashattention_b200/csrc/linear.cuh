@@ -50,17 +50,25 @@ struct GemmShape {
 //     rows (its TMEM lane). It reads 128 accumulator columns per tensor-memory
 //     wait (32 columns per wait left the epilogue slower than the products),
 //     adds the bias (one broadcast load per 8 columns), rounds to bf16 (or
-//     fp16 for columns at or beyond `f16_from`) and stores 16-byte pieces of
-//     its row; then it arrives (remotely, from CTA 1) on CTA 0's `acc_empty`.
+//     fp16 for columns at or beyond `f16_from`) and writes its row's 64-column
+//     pieces into one of the warp's two staging tiles; lane 0 stores each
+//     32 x 64 tile with a TMA bulk store. Then the warp arrives (remotely,
+//     from CTA 1) on CTA 0's `acc_empty`.
 //     No barrier other than the bounded mbarrier waits joins the epilogue
 //     warps, so a wait that gives up cannot strand the others.
 constexpr int kPairBM = 256, kPairBN = 256;
 constexpr int kPairStages = 6;
 constexpr uint32_t kPairHalfBytes = 128 * kBK * 2;  // 16 KiB: a half tile of A or of W
 
+constexpr int kEpiWarps = 4;
+constexpr uint32_t kStageTileBytes = 32 * 128;  // 32 rows x 64 columns of 16-bit y
+
 struct alignas(1024) PairSmem {
   uint8_t a[kPairStages][kPairHalfBytes];
   uint8_t b[kPairStages][kPairHalfBytes];
+  // [epilogue warp][buffer]: 32 rows x 64 columns of y (128-byte swizzle) on
+  // their way to global memory by TMA.
+  uint8_t ystage[kEpiWarps][2][kStageTileBytes];
   uint64_t full[kPairStages], empty[kPairStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
@@ -76,8 +84,9 @@ __host__ __device__ __forceinline__ int num_pair_tiles(const GemmShape& g) {
 
 __global__ void __launch_bounds__(kThreads, 1)
 linear_pair_kernel(const __grid_constant__ CUtensorMap map_a,
-                   const __grid_constant__ CUtensorMap map_w, const uint16_t* __restrict__ bias,
-                   uint16_t* __restrict__ y, const GemmShape g) {
+                   const __grid_constant__ CUtensorMap map_w,
+                   const __grid_constant__ CUtensorMap map_y, const uint16_t* __restrict__ bias,
+                   const GemmShape g) {
   extern __shared__ uint8_t smem_raw[];
   PairSmem& sm = *reinterpret_cast<PairSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -181,8 +190,8 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap map_a,
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
-    const int r = q * 32 + lane;            // row within this CTA's half of the tile
-    uint32_t lt = 0;
+    const int ew = warp - kEpiWarp0;        // this warp's staging buffers
+    uint32_t lt = 0, st_cnt = 0;
     bool ok = true;
     for (int t = cid; ok && t < n_tiles; t += n_clusters, ++lt) {
       const int tm = t / tiles_n, tn = t % tiles_n;
@@ -192,9 +201,9 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap map_a,
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int row = tm * kPairBM + static_cast<int>(rank) * 128 + r;
+      // This warp's 32 rows of the tile; rows past M are clipped by the store.
+      const int row0 = tm * kPairBM + static_cast<int>(rank) * 128 + q * 32;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kPairBN;
-      uint16_t* yrow = y + static_cast<size_t>(row) * g.N;
 #pragma unroll 1
       for (int c4 = 0; c4 < kPairBN / 128; ++c4) {
         uint32_t vv[4][32];
@@ -202,35 +211,47 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap map_a,
         for (int c1 = 0; c1 < 4; ++c1) tmem_ld32(taddr + 128 * c4 + 32 * c1, vv[c1]);
         tmem_wait_ld();
 #pragma unroll
-        for (int c1 = 0; c1 < 4; ++c1) {
-        const uint32_t (&v)[32] = vv[c1];
-        const int col0 = n0 + 128 * c4 + 32 * c1;
-        if (row < g.M) {
+        for (int hh = 0; hh < 2; ++hh) {  // 64-column halves: one staged box each
+          const int col0 = n0 + 128 * c4 + 64 * hh;
+          if (col0 >= g.N) continue;  // N is a multiple of 64
+          uint8_t* sb = sm.ystage[ew][st_cnt & 1];
+          // The store that last read this buffer has finished reading it.
+          if (lane == 0 && st_cnt >= 2) bulk_wait_group_read1();
+          __syncwarp();
           const bool f16 = col0 >= g.f16_from;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int col = col0 + 8 * u;
-            if (col < g.N) {
-              // Every lane reads the same 8 bias values: one broadcast load.
-              const uint4 bv = *reinterpret_cast<const uint4*>(bias + col);
-              const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-              uint32_t w[4];
+          for (int j = 0; j < 8; ++j) {  // 16-byte chunk j: columns col0 + 8j .. + 8
+            const uint32_t (&v)[32] = vv[2 * hh + (j >> 2)];
+            const int u = j & 3;
+            // Every lane reads the same 8 bias values: one broadcast load.
+            const uint4 bv = *reinterpret_cast<const uint4*>(bias + col0 + 8 * j);
+            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+            uint32_t w[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float a0 = __uint_as_float(v[8 * u + 2 * e]) + __uint_as_float(bw[e] << 16);
-                const float a1 = __uint_as_float(v[8 * u + 2 * e + 1]) + __uint_as_float(bw[e] & 0xFFFF0000u);
-                w[e] = f16 ? pack_f16(a0, a1) : pack_bf16(a0, a1);
-              }
-              *reinterpret_cast<uint4*>(yrow + col) = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int e = 0; e < 4; ++e) {
+              const float a0 = __uint_as_float(v[8 * u + 2 * e]) + __uint_as_float(bw[e] << 16);
+              const float a1 = __uint_as_float(v[8 * u + 2 * e + 1]) + __uint_as_float(bw[e] & 0xFFFF0000u);
+              w[e] = f16 ? pack_f16(a0, a1) : pack_bf16(a0, a1);
             }
+            *reinterpret_cast<uint4*>(sb + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
           }
-        }
+          fence_proxy_async_smem();  // generic-proxy writes, read by the TMA engine
+          __syncwarp();
+          if (lane == 0 && row0 < g.M) {  // a box wholly past M is not issued
+            tma_store_2d(&map_y, sb, col0, row0);
+            bulk_commit_group();
+          }
+          ++st_cnt;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * buf);
     }
+    // Every store this warp issued has completed before the CTA exits.
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
   }
 
   tc_fence_before();
