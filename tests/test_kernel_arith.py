@@ -73,39 +73,62 @@ def _bf16_rne(x):
 
 def pack_f16_nonneg_model(p):
     """float32/uint32 restatement of pack_f16_nonneg for one value: times
-    2^-112, add 0x1000 to the bits, keep bits [13, 29)."""
+    kF32ToF16Scale in fp32, keep bits [13, 29) of the product."""
     s = _const("kF32ToF16Scale")
     m = (np.asarray(p, dtype=np.float32) * s).astype(np.float32)
-    b = (m.view(np.uint32).astype(np.uint64) + 0x1000) >> 13
+    b = m.view(np.uint32).astype(np.uint64) >> 13
     assert np.all(b < 0x8000)   # no carry into the other half of the pair
     return b.astype(np.uint16).view(np.float16)
 
 
-def test_f16_pack_scale_is_two_to_minus_112():
-    assert float(_const("kF32ToF16Scale")) == 2.0 ** -112
+def test_f16_pack_scale():
+    # 2^-112 moves the exponent bias from 127 to 15; (1 + 3 * 2^-13) is the
+    # rounding bias, exact in fp32.
+    assert float(_const("kF32ToF16Scale")) == 2.0 ** -112 * (1 + 3 * 2.0 ** -13)
 
 
-def test_f16_pack_rounds_to_nearest_ties_away():
-    # Probabilities in [0, 2^8] (the stale-max bound). In fp16's normal range
-    # the 2^-112 multiply is exact, so the result is the correctly rounded
-    # value except that exact ties go up. Below 2^-14 the product is an fp32
-    # denormal, itself rounded to a 2^-37 grid (in p's units) first: the
-    # result is then within half an fp16 ulp plus 2^-37.
+def _fp16_neighbours(x):
+    """The fp16 values just below-or-at and just above x (x >= 2^-14, normal)."""
+    x = np.asarray(x, np.float64)
+    ulp = 2.0 ** (np.floor(np.log2(x)) - 10)
+    lo = np.floor(x / ulp) * ulp
+    return lo, lo + ulp, ulp
+
+
+def test_f16_pack_rounds_faithfully_with_the_stated_threshold():
+    # Probabilities in [2^-14, 2^8] (fp16 normals; 2^8 is the stale-max bound).
     rng = np.random.default_rng(0)
-    p = np.concatenate([rng.uniform(0, 256, 200_000), rng.uniform(0, 2.0 ** -13, 50_000),
-                        np.array([0.0, 2.0 ** -24, 2.0 ** -14, 1.0, 255.875, 256.0])]).astype(np.float32)
+    p = np.exp2(rng.uniform(-14, 8, 400_000)).astype(np.float32)
     got = pack_f16_nonneg_model(p).astype(np.float64)
-    exact = p.astype(np.float64)
-    ne = exact.astype(np.float16).astype(np.float64)          # round to nearest even
-    up = np.nextafter(ne.astype(np.float16), np.float16(np.inf)).astype(np.float64)
-    tie = np.abs(exact - ne) == np.abs(up - exact)
-    normal = exact >= 2.0 ** -14
-    assert np.all(got[normal & ~tie] == ne[normal & ~tie])
-    assert np.all(got[normal & tie] == np.maximum(ne[normal & tie], up[normal & tie]))
-    assert np.all(np.abs(got[~normal] - exact[~normal]) <= 2.0 ** -25 + 2.0 ** -37)
-    # Ties themselves: k + 1/2 fp16 ulps at 1.0 (ulp 2^-10) round up.
-    t = np.float32(1.0 + 2.0 ** -11)
-    assert float(pack_f16_nonneg_model(t)) == 1.0 + 2.0 ** -10
+    x = p.astype(np.float64)
+    lo, hi, ulp = _fp16_neighbours(x)
+    # One of the two fp16 values around p, error below 3/4 of a unit.
+    assert np.all((got == lo) | (got == hi))
+    assert np.all(np.abs(got - x) <= 0.75 * ulp)
+    # Up exactly when the dropped part exceeds 1 - 3f/8 units, f the
+    # significand (checked away from the threshold, where the fp32 product's
+    # own rounding cannot decide).
+    f = x / (2.0 ** np.floor(np.log2(x)))
+    frac = (x - lo) / ulp
+    thr = 1.0 - 3.0 * f / 8.0
+    clear = np.abs(frac - thr) > 2.0 ** -8
+    assert np.all(got[clear] == np.where(frac[clear] > thr[clear], hi[clear], lo[clear]))
+    # fp16 values stay themselves.
+    exact = np.exp2(rng.uniform(-14, 8, 10_000)).astype(np.float16).astype(np.float32)
+    assert np.array_equal(pack_f16_nonneg_model(exact).astype(np.float32), exact)
+    # The mean error over p log-uniform across the range: 3/8 E[f] - 1/2 =
+    # 3 / (8 ln 2) - 1/2 = +0.041 of a unit (plain truncation gives -1/2).
+    assert abs(np.mean((got - x) / ulp) - (3 / (8 * np.log(2)) - 0.5)) < 0.005
+
+
+def test_f16_pack_below_the_normal_range():
+    # Below 2^-14 the fp32 product is denormal: the result stays within one
+    # fp16 subnormal unit (2^-24) of p, and 0 maps to 0.
+    rng = np.random.default_rng(1)
+    p = np.concatenate([rng.uniform(0, 2.0 ** -14, 50_000), [0.0, 2.0 ** -24]]).astype(np.float32)
+    got = pack_f16_nonneg_model(p).astype(np.float64)
+    assert np.all(np.abs(got - p.astype(np.float64)) < 2.0 ** -24)
+    assert float(pack_f16_nonneg_model(np.float32(0.0))) == 0.0
 
 
 def split3_bf16_model(v):

@@ -5,8 +5,9 @@ The model follows the kernel step by step for one head: S = Q K^T in fp32
 from bf16 inputs; per 128-key tile, the row max with the stale-max rule
 (raised only when it grows by more than 2^8 in base 2), p = 2^(s*c - m*c)
 with every 6th pair of columns on the FMA-pipe polynomial, the row sum in the
-kernel's order, P packed to fp16 (round half up) and multiplied with V
-converted to fp16 (the integer conversion: exact down to 2^-14), O rescaled when the max is raised; at the end
+kernel's order, P packed to fp16 (the biased truncation of pack_f16_nonneg)
+and multiplied with V converted to fp16 (the integer conversion: exact down
+to 2^-14), O rescaled when the max is raised; at the end
 out = bf16(O / l) and lse = ln2 * (m*c + log2 l). Replacing the fp16 P and V
 with bf16 shows what the precision choice buys.
 """
