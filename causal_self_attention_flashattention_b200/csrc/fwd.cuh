@@ -10,13 +10,16 @@
 //   * Warp 8 (TMA): loads the two Q tiles once per item (double-buffered
 //     across items) and streams the 128-row K and V tiles j = 0..2p+1 through a
 //     4-stage shared-memory ring.
-//   * Warps 9 and 10 (MMA, one thread each, one per query tile q): S_q = Q_q
-//     K_j^T (M128 N128 K64) into tensor memory, issued for key tile j+1 as soon
+//   * Warps 9 and 10 (MMA, one thread each, one per warpgroup q): S_q = Q K_j^T
+//     (M128 N128 K64) into tensor memory, issued for key tile j+1 as soon
 //     as the softmax has read S_q(j), then O_q += P_q V_j (M128 N64 K128) with
 //     P_q read from tensor memory. Key tiles above the diagonal are never
-//     issued. Each query tile has its own issuing thread, so neither waits on
-//     the other tile's softmax.
-//   * Warps 0-7 (softmax): two warpgroups, warpgroup q serves query tile q.
+//     issued. Each warpgroup has its own issuing thread, so neither waits on
+//     the other's softmax.
+//   * Warps 0-7 (softmax): two warpgroups. Warpgroup q serves query tile q of
+//     the CTA's even items and tile 1 - q of its odd ones: tile i0 + 1 takes
+//     one key tile more, and alternating it keeps one warpgroup from doing
+//     every item's extra step while the other idles.
 //     Each thread owns one query row (its TMEM lane) and all 128 columns of
 //     every key tile: it loads the row of S from tensor memory, applies the
 //     causal mask on the diagonal tile, runs the online softmax in base 2
@@ -32,8 +35,9 @@
 //     3e-8); a v that is not finite with |v| <= 65504 is reported in the
 //     status word.
 //
-// Tensor memory (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256),
-// P_0 [256,320), P_1 [320,384) (fp16 pairs), O_0 [384,448), O_1 [448,512).
+// Tensor memory (512 columns x 128 lanes, fp32; index = warpgroup): S_0
+// [0,128), S_1 [128,256), P_0 [256,320), P_1 [320,384) (fp16 pairs), O_0
+// [384,448), O_1 [448,512).
 
 #pragma once
 
@@ -47,8 +51,8 @@ constexpr int kStages = 4;
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;       // issues for query tile 0, owns the TMEM allocation
-constexpr int kMmaWarp1 = 10;     // issues for query tile 1
+constexpr int kMmaWarp = 9;       // issues for warpgroup 0, owns the TMEM allocation
+constexpr int kMmaWarp1 = 10;     // issues for warpgroup 1
 constexpr int kConvertWarp = 11;
 // Register split (setmaxnreg): the TMA/MMA/convert warpgroup (warps 8-11) gives
 // registers to the two softmax warpgroups, which hold a whole 128-column row
@@ -74,6 +78,21 @@ __device__ __forceinline__ uint32_t col_o(int q) { return 384 + q * 64; }
 // Bytes of one 128 x 64 Q or K tile: bf16, or e4m3 in the FP8 forward.
 template <bool kFp8>
 constexpr int kQKBytes = kFp8 ? kTileBytes / 2 : kTileBytes;
+
+// The deal of items to CTAs for one launch, computed on the host and passed
+// by value (a kernel parameter): CTA c runs items base + item[t] for t in
+// [start[c], start[c + 1]), in that order, at most kSchedSlots of them. The
+// host fills it longest-processing-time first (items in decode_item order,
+// heaviest first, each to the CTA with the least work so far) and splits a
+// forward whose items do not fit one table into several launches.
+constexpr int kSchedMaxCtas = 160;
+constexpr int kSchedMaxItems = 6144;
+constexpr int kSchedSlots = 64;
+struct ItemSchedule {
+  int base;
+  uint16_t start[kSchedMaxCtas + 1];
+  uint16_t item[kSchedMaxItems];
+};
 
 template <bool kFp8>
 struct alignas(1024) Smem {
@@ -109,6 +128,14 @@ __device__ __forceinline__ Item decode_item(int k, const AttnShape& sh) {
   it.has1 = (2 * p + 1) < n_qt;
   it.n_kv = it.has1 ? 2 * p + 2 : 2 * p + 1;
   return it;
+}
+
+// The query tile of an item (0: i0, 1: i0 + 1) that warpgroup / issuer q
+// serves in the CTA's it_cnt-th item. Tile i0 + 1 sees one key tile more, so
+// the two swap on every other item: otherwise warpgroup 1 would take that
+// extra step in every item and set the CTA's time alone.
+__device__ __forceinline__ int item_tile(int q, uint32_t it_cnt) {
+  return q ^ static_cast<int>(it_cnt & 1);
 }
 
 __host__ __device__ __forceinline__ int num_items(const AttnShape& sh) {
@@ -153,7 +180,8 @@ template <bool kFp8, bool kV16 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
                 const __grid_constant__ CUtensorMap map_v8, __nv_bfloat16* __restrict__ out,
-                float* __restrict__ lse, const AttnShape sh, const float* __restrict__ dequant) {
+                float* __restrict__ lse, const AttnShape sh, const float* __restrict__ dequant,
+                const __grid_constant__ ItemSchedule sched) {
   static_assert(!(kFp8 && kV16), "the FP8 forward widens its own e4m3 V");
   constexpr int kQK = kQKBytes<kFp8>;
   extern __shared__ uint8_t smem_raw[];
@@ -164,6 +192,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
   const int C = sh.H * kD;
   const int n_items = num_items(sh);
   volatile int* abort = &sm.abort;
+
+  // This CTA's items, in order, and their count in the last slot (the
+  // __syncthreads below publishes them to every role).
+  __shared__ int items[kSchedSlots + 1];
+  {
+    const int t0 = sched.start[blockIdx.x];
+    const int n = min(sched.start[blockIdx.x + 1] - t0, kSchedSlots);
+    if (threadIdx.x == 0) items[kSchedSlots] = n;
+    for (int t = threadIdx.x; t < n; t += blockDim.x) items[t] = sched.base + sched.item[t0 + t];
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -204,8 +242,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
     // ------------------------------------------------------------ TMA warp
     if (lane == 0) {
       uint32_t kv_it = 0, it_cnt = 0;
-      for (int rnd = 0; rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
-        const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+      for (int rnd = 0; rnd < items[kSchedSlots]; ++rnd) {
+        const int k = items[rnd];
         if (k >= n_items) continue;
         const Item it = decode_item(k, sh);
         const int slot = it_cnt & 1;
@@ -244,7 +282,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
     __syncwarp();
   } else if (warp == kMmaWarp || warp == kMmaWarp1) {
     // ------------------------------------------------------------ MMA warps
-    // One issuing thread per query tile q. Per item: S_q(0); then for each
+    // One issuing thread per warpgroup q, for query tile item_tile(q, item)
+    // of each item. Per item: S_q(0); then for each
     // key tile j the thread issues S_q(j+1) once the softmax has read S_q(j),
     // then O_q += P_q(j) V_j once P_q(j) is written and V_j converted.
     const int q = warp - kMmaWarp;
@@ -255,14 +294,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
       const uint32_t t_s = tmem + col_s(q), t_p = tmem + col_p(q), t_o = tmem + col_o(q);
       uint32_t kv_it = 0, it_cnt = 0, s_cnt = 0, p_cnt = 0;
       bool ok = true;
-      for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
-        const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+      for (int rnd = 0; ok && rnd < items[kSchedSlots]; ++rnd) {
+        const int k = items[rnd];
         if (k >= n_items) continue;
         const Item it = decode_item(k, sh);
         const int slot = it_cnt & 1;
+        const int tq = item_tile(q, it_cnt);
         // Key tiles this query tile sees, and those the other one sees.
-        const int n = q == 0 ? it.i0 + 1 : (it.has1 ? it.i0 + 2 : 0);
-        const int n_other = q == 0 ? (it.has1 ? it.i0 + 2 : 0) : it.i0 + 1;
+        const int n = tq == 0 ? it.i0 + 1 : (it.has1 ? it.i0 + 2 : 0);
+        const int n_other = tq == 0 ? (it.has1 ? it.i0 + 2 : 0) : it.i0 + 1;
         if (n == 0) {
           // No second query tile in this item: this thread still releases its
           // share of the Q slot, after the slot's previous phase is complete
@@ -279,8 +319,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
         } else {
           if (!mbar_wait(&sm.q_full[slot], (it_cnt >> 1) & 1, kSiteFwdMma, abort)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t qdesc = kFp8 ? smem_desc_sw64(smem_u32(sm.q[slot][q]), 512)
-                                      : smem_desc_sw128(smem_u32(sm.q[slot][q]), 16, 1024);
+          const uint64_t qdesc = kFp8 ? smem_desc_sw64(smem_u32(sm.q[slot][tq]), 512)
+                                      : smem_desc_sw128(smem_u32(sm.q[slot][tq]), 16, 1024);
           // S_q(jj) = Q_q K(jj)^T. bf16: K = 64 in four steps of 16 (32 bytes
           // each); e4m3: two steps of 32 (32 bytes each).
           auto issue_s = [&](int jj) -> bool {
@@ -340,8 +380,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
     // ------------------------------------------------------------ convert V
     uint32_t kv_it = 0;
     bool ok = true;
-    for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
-      const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+    for (int rnd = 0; ok && rnd < items[kSchedSlots]; ++rnd) {
+      const int k = items[rnd];
       if (k >= n_items) continue;
       const Item it = decode_item(k, sh);
       for (int j = 0; j < it.n_kv; ++j, ++kv_it) {
@@ -405,7 +445,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
     // end (both fold in the dequantisation of e4m3 inputs).
     const float c_log2 = kFp8 ? sh.scale_log2 * dequant[0] * dequant[1] : sh.scale_log2;
     const float o_mul = kFp8 ? 256.f * dequant[2] : 1.f;
-    const int q = warp >> 2;                       // query tile of the pair
+    const int q = warp >> 2;                       // warpgroup; its query tile is item_tile()
     const int r = ((warp & 3) << 5) + lane;        // row within the tile = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
     const uint32_t t_s = tmem + lane_base + col_s(q);
@@ -420,12 +460,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
     int p_b = 0, p_h = 0, p_row = 0;
     float p_m = 0.f, p_l = 0.f;
     bool ok = true;
-    for (int rnd = 0; ok && rnd * static_cast<int>(gridDim.x) < n_items; ++rnd) {
-      const int k = snake_item(rnd, gridDim.x, blockIdx.x);
+    uint32_t it_cnt = 0;
+    for (int rnd = 0; ok && rnd < items[kSchedSlots]; ++rnd) {
+      const int k = items[rnd];
       if (k >= n_items) continue;
       const Item it = decode_item(k, sh);
-      if (q == 1 && !it.has1) continue;
-      const int i = it.i0 + q;
+      const int tq = item_tile(q, it_cnt++);
+      if (tq == 1 && !it.has1) continue;
+      const int i = it.i0 + tq;
       const int row = i * kBlockM + r;
       // Running max m (raw logit units, as read from S) and running sum l of
       // 2^(s*c - m*c), c = c_log2. m is only raised when the row max

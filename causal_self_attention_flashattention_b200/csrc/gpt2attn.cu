@@ -11,10 +11,14 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <queue>
+#include <utility>
+#include <vector>
 
 #include "gpt2attn.h"
 #include "checks.h"
@@ -327,6 +331,106 @@ ga::AttnShape make_shape(int B, int T, int H, float scale) {
 
 int grid_for(int items, int num_sms) { return items < num_sms ? items : num_sms; }
 
+// The forward's deal of items to CTAs (ga::fwd::ItemSchedule), longest
+// processing time first. Items come heaviest first (the order of
+// decode_item); each goes to the CTA with the least work so far, the lowest
+// index on ties. An item with n key tiles costs 2n + kItemStartCost2 in
+// half-tile steps: the constant stands for what an item costs beyond its
+// tiles (its first S product, the previous item's output, the swap of the
+// two warpgroups' tiles), about two and a half tile steps when measured
+// (A/B of 0, 1.26 and 2.5 at B=16 T=1024 H=12; 2.5 was fastest).
+constexpr long kItemStartCost2 = 5;
+
+// Deals items [k0, k1) to `grid` CTAs into *s. False if a CTA would get more
+// than kSchedSlots items (the caller then deals fewer items per launch).
+bool build_fwd_schedule(ga::fwd::ItemSchedule* s, int n_qt, int bh, long k0, long k1, int grid) {
+  const int n_pairs = (n_qt + 1) / 2;
+  const long n = k1 - k0;
+  if (grid <= 0 || grid > ga::fwd::kSchedMaxCtas || n <= 0 || n > ga::fwd::kSchedMaxItems)
+    return false;
+  using Load = std::pair<long, int>;  // (work so far, CTA)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < grid; ++c) heap.push(Load(0, c));
+  std::vector<int> owner(n), count(grid, 0);
+  for (long k = k0; k < k1; ++k) {
+    const int p = n_pairs - 1 - static_cast<int>(k / bh);
+    const int n_kv = (2 * p + 1) < n_qt ? 2 * p + 2 : 2 * p + 1;
+    const Load least = heap.top();
+    heap.pop();
+    owner[k - k0] = least.second;
+    if (++count[least.second] > ga::fwd::kSchedSlots) return false;
+    heap.push(Load(least.first + 2L * n_kv + kItemStartCost2, least.second));
+  }
+  int off = 0;
+  for (int c = 0; c < grid; ++c) {
+    s->start[c] = static_cast<uint16_t>(off);
+    off += count[c];
+    count[c] = s->start[c];  // next free place in CTA c's list
+  }
+  s->start[grid] = static_cast<uint16_t>(off);
+  for (long t = 0; t < n; ++t) s->item[count[owner[t]]++] = static_cast<uint16_t>(t);
+  s->base = static_cast<int>(k0);
+  return true;
+}
+
+// Calls launch(schedule, grid) once per launch of a forward over B*H heads
+// and T rows on num_sms SMs, in item order. One launch unless the items do
+// not fit one table. The deal of a one-launch forward is cached per (query
+// tiles, heads, SMs) in a fixed table replaced round-robin under its own
+// mutex. Returns false if a launch failed (launch() returned false).
+struct SchedCacheEntry {
+  bool used = false;
+  int n_qt = 0, bh = 0, num_sms = 0;
+  ga::fwd::ItemSchedule sched;
+  int grid = 0;
+};
+constexpr int kSchedCacheSize = 8;
+std::mutex g_sched_mutex;
+SchedCacheEntry g_sched_cache[kSchedCacheSize];
+int g_sched_next = 0;
+
+template <class Launch>
+bool for_each_fwd_launch(int B, int T, int H, int num_sms, Launch launch) {
+  const int n_qt = (T + ga::kBlockM - 1) / ga::kBlockM, bh = B * H;
+  const long items = static_cast<long>(bh) * ((n_qt + 1) / 2);
+  ga::fwd::ItemSchedule sched;
+  int cached_grid = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_sched_mutex);
+    for (const SchedCacheEntry& e : g_sched_cache)
+      if (e.used && e.n_qt == n_qt && e.bh == bh && e.num_sms == num_sms) {
+        sched = e.sched;
+        cached_grid = e.grid;
+        break;
+      }
+  }
+  if (cached_grid > 0) return launch(sched, cached_grid);
+  long chunk = ga::fwd::kSchedMaxItems;
+  for (long k0 = 0; k0 < items;) {
+    const long k1 = std::min(items, k0 + chunk);
+    const int grid = static_cast<int>(
+        std::min<long>(k1 - k0, std::min(num_sms, ga::fwd::kSchedMaxCtas)));
+    if (!build_fwd_schedule(&sched, n_qt, bh, k0, k1, grid)) {
+      chunk /= 2;  // fits at the latest once chunk <= kSchedSlots
+      continue;
+    }
+    if (k0 == 0 && k1 == items) {
+      std::lock_guard<std::mutex> lock(g_sched_mutex);
+      SchedCacheEntry& e = g_sched_cache[g_sched_next];
+      g_sched_next = (g_sched_next + 1) % kSchedCacheSize;
+      e.sched = sched;
+      e.grid = grid;
+      e.n_qt = n_qt;
+      e.bh = bh;
+      e.num_sms = num_sms;
+      e.used = true;
+    }
+    if (!launch(sched, grid)) return false;
+    k0 = k1;
+  }
+  return true;
+}
+
 size_t delta_bytes(int B, int T, int H) {
   const size_t n = static_cast<size_t>(B) * H * T * sizeof(float);
   return (n + 255) & ~static_cast<size_t>(255);
@@ -355,17 +459,19 @@ ga_status launch_fwd(const void* qkv, void* out, float* lse, int B, int T, int H
   CUtensorMap map_qkv;
   if (!make_map(&map_qkv, qkv, static_cast<uint64_t>(3) * H * kD, T, B)) return GA_ERR_CUDA;
   const ga::AttnShape sh = make_shape(B, T, H, scale);
-  const int items = ga::fwd::num_items(sh);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (v16)
-    ga::fwd::attn_fwd_kernel<false, true><<<grid_for(items, info->num_sms), ga::fwd::kThreads,
-                                            ga::fwd::kSmemBytes<false>, s>>>(
-        map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr);
-  else
-    ga::fwd::attn_fwd_kernel<false><<<grid_for(items, info->num_sms), ga::fwd::kThreads,
-                                      ga::fwd::kSmemBytes<false>, s>>>(
-        map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr);
-  return check_launch();
+  ga_status ls = GA_OK;
+  for_each_fwd_launch(B, T, H, info->num_sms, [&](const ga::fwd::ItemSchedule& sched, int grid) {
+    if (v16)
+      ga::fwd::attn_fwd_kernel<false, true><<<grid, ga::fwd::kThreads,
+                                              ga::fwd::kSmemBytes<false>, s>>>(
+          map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr, sched);
+    else
+      ga::fwd::attn_fwd_kernel<false><<<grid, ga::fwd::kThreads, ga::fwd::kSmemBytes<false>, s>>>(
+          map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr, sched);
+    return (ls = check_launch()) == GA_OK;
+  });
+  return ls;
 }
 
 }  // namespace
@@ -418,13 +524,15 @@ ga_status gpt2_attn_fwd_fp8(const void* qkv8, const float* scales, void* out, fl
   if (!make_map_u8(&map_qk, qkv8, inner, T, B, CU_TENSOR_MAP_SWIZZLE_64B)) return GA_ERR_CUDA;
   if (!make_map_u8(&map_v, qkv8, inner, T, B, CU_TENSOR_MAP_SWIZZLE_NONE)) return GA_ERR_CUDA;
   const ga::AttnShape sh = make_shape(B, T, H, scale);
-  const int items = ga::fwd::num_items(sh);
-  ga::fwd::attn_fwd_kernel<true><<<grid_for(items, info->num_sms), ga::fwd::kThreads,
-                                   ga::fwd::kSmemBytes<true>,
-                                   reinterpret_cast<cudaStream_t>(stream)>>>(
-      map_qk, map_v, static_cast<__nv_bfloat16*>(out), lse, sh,
-      scales + ga::fp8::kDequantOffset);
-  return check_launch();
+  ga_status ls = GA_OK;
+  for_each_fwd_launch(B, T, H, info->num_sms, [&](const ga::fwd::ItemSchedule& sched, int grid) {
+    ga::fwd::attn_fwd_kernel<true><<<grid, ga::fwd::kThreads, ga::fwd::kSmemBytes<true>,
+                                     reinterpret_cast<cudaStream_t>(stream)>>>(
+        map_qk, map_v, static_cast<__nv_bfloat16*>(out), lse, sh,
+        scales + ga::fp8::kDequantOffset, sched);
+    return (ls = check_launch()) == GA_OK;
+  });
+  return ls;
 }
 
 ga_status gpt2_attn_bwd_workspace_size(int B, int T, int H, int D, size_t* bytes) {
@@ -760,5 +868,28 @@ const char* gpt2_attn_status_string(ga_status s) {
 }
 
 int gpt2_attn_version(void) { return 100; }
+
+int gpt2_attn_fwd_item_schedule(int B, int T, int H, int num_sms, int* launch, int* cta,
+                                int* pos, long n) {
+  if (launch == nullptr || cta == nullptr || pos == nullptr || B <= 0 || T <= 0 || H <= 0 ||
+      num_sms <= 0)
+    return -GA_ERR_INVALID_ARG;
+  const int n_qt = (T + ga::kBlockM - 1) / ga::kBlockM;
+  const long items = static_cast<long>(B) * H * ((n_qt + 1) / 2);
+  if (n < items || items > INT32_MAX) return -GA_ERR_INVALID_ARG;
+  int n_launch = 0;
+  for_each_fwd_launch(B, T, H, num_sms, [&](const ga::fwd::ItemSchedule& sched, int grid) {
+    for (int c = 0; c < grid; ++c)
+      for (int t = sched.start[c]; t < sched.start[c + 1]; ++t) {
+        const long k = sched.base + static_cast<long>(sched.item[t]);
+        launch[k] = n_launch;
+        cta[k] = c;
+        pos[k] = t - sched.start[c];
+      }
+    ++n_launch;
+    return true;
+  });
+  return n_launch;
+}
 
 }  // extern "C"

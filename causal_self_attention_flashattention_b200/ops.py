@@ -57,6 +57,7 @@ EXPORTED_SYMBOLS = (
     "gpt2_attn_out_proj",
     "gpt2_attn_status_string",
     "gpt2_attn_version",
+    "gpt2_attn_fwd_item_schedule",
 )
 
 _vp = ctypes.c_void_p
@@ -112,6 +113,9 @@ _lib.gpt2_attn_status_string.argtypes = [_i]
 _lib.gpt2_attn_status_string.restype = ctypes.c_char_p
 _lib.gpt2_attn_version.argtypes = []
 _lib.gpt2_attn_version.restype = _i
+_ip = ctypes.POINTER(ctypes.c_int)
+_lib.gpt2_attn_fwd_item_schedule.argtypes = [_i, _i, _i, _i, _ip, _ip, _ip, ctypes.c_long]
+_lib.gpt2_attn_fwd_item_schedule.restype = _i
 
 
 class AttnError(RuntimeError):
@@ -132,6 +136,22 @@ def status_string(status: int) -> str:
 
 def version() -> int:
     return int(_lib.gpt2_attn_version())
+
+
+def fwd_item_schedule(B: int, T: int, H: int, num_sms: int):
+    """The forward's deal of items to launches and CTAs for (B, T, H) on
+    num_sms SMs (host code, no GPU needed): int32 arrays (launch, cta, pos)
+    indexed by item, and the number of launches. Raises ValueError on bad
+    arguments."""
+    import numpy as np
+
+    n_items = B * H * (((T + 127) // 128 + 1) // 2) if min(B, T, H) > 0 else 1
+    arrs = [np.full(n_items, -1, dtype=np.int32) for _ in range(3)]
+    ptrs = [a.ctypes.data_as(_ip) for a in arrs]
+    n = _lib.gpt2_attn_fwd_item_schedule(B, T, H, num_sms, *ptrs, n_items)
+    if n < 0:
+        raise ValueError(f"gpt2_attn_fwd_item_schedule: {status_string(-n)}")
+    return arrs[0], arrs[1], arrs[2], n
 
 
 def _check(status: int, where: str) -> None:

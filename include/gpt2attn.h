@@ -326,6 +326,28 @@ ga_status gpt2_attn_selftest_wait_timeout(unsigned long long limit_ns,
                                           gpt2attn_stream_t stream);
 
 /*
+ * The forward's deal of work items to CTAs and launches, as gpt2_attn_fwd,
+ * _fwd_v16 and _fwd_fp8 make it for (B, T, H) on a device with num_sms SMs.
+ * An item is one (b, h) and a pair of adjacent 128-row query tiles; there are
+ * n_items = B*H*ceil(ceil(T/128)/2) of them, numbered heaviest first (item k
+ * covers query tiles 2p and 2p + 1, p = ceil(ceil(T/128)/2) - 1 - k / (B*H),
+ * of head (b, h) = divmod(k % (B*H), H)). The items are split into launches
+ * of consecutive items (one launch unless they exceed one kernel parameter
+ * table: 6144 items, 64 per CTA), each on min(its items, num_sms, 160) CTAs.
+ * Within a launch every item goes, in order, to the CTA with the least work
+ * so far (longest processing time first; an item of n key tiles counts
+ * n + 2.5 tile steps). For every item k, launch[k] receives its launch,
+ * cta[k] the CTA that runs it and pos[k] its place in that CTA's list (a CTA
+ * runs its items in increasing pos). `n` is the capacity of the three arrays
+ * (>= n_items). Returns the number of launches, or -GA_ERR_INVALID_ARG on a
+ * null pointer, a non-positive size or n < n_items. Host code only: no CUDA
+ * call, usable without a GPU. The deal changes which CTA computes an item,
+ * never what it computes.
+ */
+int gpt2_attn_fwd_item_schedule(int B, int T, int H, int num_sms, int* launch, int* cta,
+                                int* pos, long n);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word.
  * Returns GA_ERR_TIMEOUT if a kernel of this library gave up on a device-side
  * wait since the last call (the kernel then stopped early and its outputs are

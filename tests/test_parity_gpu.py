@@ -149,6 +149,30 @@ def test_several_items_per_cta(ops, B, T, H):
     check_all(ops, B, T, H, seed=B + T + H)
 
 
+def test_forward_split_over_two_launches(ops):
+    """7000 one-tile items exceed one launch's item table (6144): the forward
+    runs items 0-6143 in one launch and 6144-6999 in a second. Heads on both
+    sides of the split, and at its edge, match the oracle."""
+    B, T, H = 7, 128, 1000
+    launch, _, _, n_launch = ops.fwd_item_schedule(B, T, H, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert n_launch == 2
+    qkv_bf, dout_bf = make_inputs(B, T, H, 64, seed=7)
+    out, lse = ops.attn_fwd(qkv_bf.cuda(), 0.125)
+    st, word = ops.last_device_status()
+    assert st == ops.GA_OK, (st, hex(word))
+    out, lse = out.cpu(), lse.cpu()
+    # item k is head (b, h) = divmod(k, H) here (one query-tile pair per head)
+    for b, hs in ((0, list(range(0, 4))), (6, list(range(140, 150))), (6, [999])):
+        assert {int(launch[b * H + h]) for h in hs} <= {0, 1}
+        sub = qkv_bf[b:b + 1, :, :, hs, :].contiguous()
+        o, l, _ = orc.attention_forward_backward(
+            sub.double().numpy(), np.zeros((1, T, len(hs), 64)), 0.125)
+        ok, err, _ = out_error_ok(out[b:b + 1, :, hs].double().numpy(), o)
+        assert ok, (b, hs, err)
+        assert np.max(np.abs(lse[b:b + 1, hs].double().numpy() - l)) <= LSE_TOL
+    assert {int(launch[6 * H + h]) for h in (140, 150)} == {0, 1}
+
+
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_small_gpt2_shape_seeds(ops, seed):
     check_all(ops, 1, 128, 12, seed=seed)
