@@ -84,14 +84,18 @@ constexpr int kQKBytes = kFp8 ? kTileBytes / 2 : kTileBytes;
 // [start[c], start[c + 1]), in that order, at most kSchedSlots of them. The
 // host fills it longest-processing-time first (items in decode_item order,
 // heaviest first, each to the CTA with the least work so far) and splits a
-// forward whose items do not fit one table into several launches.
+// forward whose items do not fit one table into several launches. Every
+// launch copies the whole parameter, so a launch of at most kSchedSmall items
+// takes the small table.
 constexpr int kSchedMaxCtas = 160;
+constexpr int kSchedSmall = 1024;
 constexpr int kSchedMaxItems = 6144;
 constexpr int kSchedSlots = 64;
+template <int kItems>
 struct ItemSchedule {
   int base;
   uint16_t start[kSchedMaxCtas + 1];
-  uint16_t item[kSchedMaxItems];
+  uint16_t item[kItems];
 };
 
 template <bool kFp8>
@@ -176,12 +180,12 @@ __device__ __forceinline__ void store_row(const uint32_t (&o)[64], int b, int h,
 // kV16: the v slot of qkv already holds fp16 (q and k stay bf16), as the
 // c_attn GEMM writes it when asked; the convert warp then only passes each V
 // tile on (kFp8 must be false).
-template <bool kFp8, bool kV16 = false>
+template <bool kFp8, bool kV16, int kSchedItems>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
                 const __grid_constant__ CUtensorMap map_v8, __nv_bfloat16* __restrict__ out,
                 float* __restrict__ lse, const AttnShape sh, const float* __restrict__ dequant,
-                const __grid_constant__ ItemSchedule sched) {
+                const __grid_constant__ ItemSchedule<kSchedItems> sched) {
   static_assert(!(kFp8 && kV16), "the FP8 forward widens its own e4m3 V");
   constexpr int kQK = kQKBytes<kFp8>;
   extern __shared__ uint8_t smem_raw[];

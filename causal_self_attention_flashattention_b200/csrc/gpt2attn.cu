@@ -78,6 +78,19 @@ void record_cuda_error(unsigned long long step, unsigned int code) {
   g_cuda_error.store((step << 32) | code, std::memory_order_relaxed);
 }
 
+// Opts one forward kernel into its dynamic shared memory and checks that it
+// was compiled for the register count its setmaxnreg split assumes.
+template <class Kernel>
+bool setup_fwd_kernel(Kernel kernel, bool fp8) {
+  const int smem = static_cast<int>(fp8 ? ga::fwd::kSmemBytes<true> : ga::fwd::kSmemBytes<false>);
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return false;
+  cudaFuncAttributes fa;
+  return cudaFuncGetAttributes(&fa, kernel) == cudaSuccess &&
+         fa.numRegs >= static_cast<int>(ga::fwd::kLaunchRegs);
+}
+
 // With g_mutex held: fills g_devices[dev] on its first use (SM count, the
 // dynamic shared-memory opt-in of every kernel). Returns nullptr on failure.
 const DeviceInfo* setup_device(int dev) {
@@ -102,30 +115,16 @@ const DeviceInfo* setup_device(int dev) {
   }
   if (cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return nullptr;
-  if (cudaFuncSetAttribute(ga::fwd::attn_fwd_kernel<false>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(ga::fwd::kSmemBytes<false>)) != cudaSuccess)
-    return nullptr;
-  if (cudaFuncSetAttribute(ga::fwd::attn_fwd_kernel<true>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(ga::fwd::kSmemBytes<true>)) != cudaSuccess)
-    return nullptr;
-  if (cudaFuncSetAttribute(ga::fwd::attn_fwd_kernel<false, true>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(ga::fwd::kSmemBytes<false>)) != cudaSuccess)
-    return nullptr;
-  // The forward kernel's setmaxnreg split (warpgroup budgets that add up to the
-  // block's allocation) is only safe if it launches with the register count
-  // the split was sized for.
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel<false>) != cudaSuccess ||
-      fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
-    return nullptr;
-  if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel<true>) != cudaSuccess ||
-      fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
-    return nullptr;
-  if (cudaFuncGetAttributes(&fa, ga::fwd::attn_fwd_kernel<false, true>) != cudaSuccess ||
-      fa.numRegs < static_cast<int>(ga::fwd::kLaunchRegs))
+  // The forward kernels (bf16, FP8, fp16-v; small and large item tables).
+  // Their setmaxnreg split (warpgroup budgets that add up to the block's
+  // allocation) is only safe if they launch with the register count the split
+  // was sized for.
+  if (!setup_fwd_kernel(ga::fwd::attn_fwd_kernel<false, false, ga::fwd::kSchedSmall>, false) ||
+      !setup_fwd_kernel(ga::fwd::attn_fwd_kernel<false, false, ga::fwd::kSchedMaxItems>, false) ||
+      !setup_fwd_kernel(ga::fwd::attn_fwd_kernel<true, false, ga::fwd::kSchedSmall>, true) ||
+      !setup_fwd_kernel(ga::fwd::attn_fwd_kernel<true, false, ga::fwd::kSchedMaxItems>, true) ||
+      !setup_fwd_kernel(ga::fwd::attn_fwd_kernel<false, true, ga::fwd::kSchedSmall>, false) ||
+      !setup_fwd_kernel(ga::fwd::attn_fwd_kernel<false, true, ga::fwd::kSchedMaxItems>, false))
     return nullptr;
 
   if (cudaFuncSetAttribute(ga::bwd::dkdv::attn_bwd_dkdv_kernel,
@@ -331,6 +330,9 @@ ga::AttnShape make_shape(int B, int T, int H, float scale) {
 
 int grid_for(int items, int num_sms) { return items < num_sms ? items : num_sms; }
 
+using FwdSchedule = ga::fwd::ItemSchedule<ga::fwd::kSchedMaxItems>;
+using FwdScheduleSmall = ga::fwd::ItemSchedule<ga::fwd::kSchedSmall>;
+
 // The forward's deal of items to CTAs (ga::fwd::ItemSchedule), longest
 // processing time first. Items come heaviest first (the order of
 // decode_item); each goes to the CTA with the least work so far, the lowest
@@ -343,7 +345,7 @@ constexpr long kItemStartCost2 = 5;
 
 // Deals items [k0, k1) to `grid` CTAs into *s. False if a CTA would get more
 // than kSchedSlots items (the caller then deals fewer items per launch).
-bool build_fwd_schedule(ga::fwd::ItemSchedule* s, int n_qt, int bh, long k0, long k1, int grid) {
+bool build_fwd_schedule(FwdSchedule* s, int n_qt, int bh, long k0, long k1, int grid) {
   const int n_pairs = (n_qt + 1) / 2;
   const long n = k1 - k0;
   if (grid <= 0 || grid > ga::fwd::kSchedMaxCtas || n <= 0 || n > ga::fwd::kSchedMaxItems)
@@ -373,7 +375,7 @@ bool build_fwd_schedule(ga::fwd::ItemSchedule* s, int n_qt, int bh, long k0, lon
   return true;
 }
 
-// Calls launch(schedule, grid) once per launch of a forward over B*H heads
+// Calls launch(schedule, grid, items) once per launch of a forward over B*H heads
 // and T rows on num_sms SMs, in item order. One launch unless the items do
 // not fit one table. The deal of a one-launch forward is cached per (query
 // tiles, heads, SMs) in a fixed table replaced round-robin under its own
@@ -381,30 +383,53 @@ bool build_fwd_schedule(ga::fwd::ItemSchedule* s, int n_qt, int bh, long k0, lon
 struct SchedCacheEntry {
   bool used = false;
   int n_qt = 0, bh = 0, num_sms = 0;
-  ga::fwd::ItemSchedule sched;
+  FwdSchedule sched;
   int grid = 0;
+  int n = 0;  // items in the launch
 };
 constexpr int kSchedCacheSize = 8;
 std::mutex g_sched_mutex;
 SchedCacheEntry g_sched_cache[kSchedCacheSize];
 int g_sched_next = 0;
 
+// Launches attn_fwd_kernel<kFp8, kV16> over the n items of `sched` on `grid`
+// CTAs, with the small item table when they fit it.
+template <bool kFp8, bool kV16, class... Args>
+void launch_fwd_kernel(const FwdSchedule& sched, int grid, int n, cudaStream_t stream,
+                       Args... args) {
+  const size_t smem = kFp8 ? ga::fwd::kSmemBytes<true> : ga::fwd::kSmemBytes<false>;
+  if (n <= ga::fwd::kSchedSmall) {
+    FwdScheduleSmall small;
+    small.base = sched.base;
+    std::copy(sched.start, sched.start + grid + 1, small.start);
+    std::copy(sched.item, sched.item + n, small.item);
+    ga::fwd::attn_fwd_kernel<kFp8, kV16, ga::fwd::kSchedSmall>
+        <<<grid, ga::fwd::kThreads, smem, stream>>>(args..., small);
+  } else {
+    ga::fwd::attn_fwd_kernel<kFp8, kV16, ga::fwd::kSchedMaxItems>
+        <<<grid, ga::fwd::kThreads, smem, stream>>>(args..., sched);
+  }
+}
+
 template <class Launch>
 bool for_each_fwd_launch(int B, int T, int H, int num_sms, Launch launch) {
   const int n_qt = (T + ga::kBlockM - 1) / ga::kBlockM, bh = B * H;
   const long items = static_cast<long>(bh) * ((n_qt + 1) / 2);
-  ga::fwd::ItemSchedule sched;
-  int cached_grid = 0;
+  FwdSchedule sched;
+  int cached_grid = 0, cached_n = 0;
   {
     std::lock_guard<std::mutex> lock(g_sched_mutex);
     for (const SchedCacheEntry& e : g_sched_cache)
       if (e.used && e.n_qt == n_qt && e.bh == bh && e.num_sms == num_sms) {
-        sched = e.sched;
         cached_grid = e.grid;
+        cached_n = e.n;
+        sched.base = e.sched.base;
+        std::copy(e.sched.start, e.sched.start + cached_grid + 1, sched.start);
+        std::copy(e.sched.item, e.sched.item + cached_n, sched.item);
         break;
       }
   }
-  if (cached_grid > 0) return launch(sched, cached_grid);
+  if (cached_grid > 0) return launch(sched, cached_grid, cached_n);
   long chunk = ga::fwd::kSchedMaxItems;
   for (long k0 = 0; k0 < items;) {
     const long k1 = std::min(items, k0 + chunk);
@@ -420,12 +445,13 @@ bool for_each_fwd_launch(int B, int T, int H, int num_sms, Launch launch) {
       g_sched_next = (g_sched_next + 1) % kSchedCacheSize;
       e.sched = sched;
       e.grid = grid;
+      e.n = static_cast<int>(k1 - k0);
       e.n_qt = n_qt;
       e.bh = bh;
       e.num_sms = num_sms;
       e.used = true;
     }
-    if (!launch(sched, grid)) return false;
+    if (!launch(sched, grid, static_cast<int>(k1 - k0))) return false;
     k0 = k1;
   }
   return true;
@@ -461,14 +487,15 @@ ga_status launch_fwd(const void* qkv, void* out, float* lse, int B, int T, int H
   const ga::AttnShape sh = make_shape(B, T, H, scale);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   ga_status ls = GA_OK;
-  for_each_fwd_launch(B, T, H, info->num_sms, [&](const ga::fwd::ItemSchedule& sched, int grid) {
+  for_each_fwd_launch(B, T, H, info->num_sms, [&](const FwdSchedule& sched, int grid, int n) {
     if (v16)
-      ga::fwd::attn_fwd_kernel<false, true><<<grid, ga::fwd::kThreads,
-                                              ga::fwd::kSmemBytes<false>, s>>>(
-          map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr, sched);
+      launch_fwd_kernel<false, true>(sched, grid, n, s, map_qkv, map_qkv,
+                                     static_cast<__nv_bfloat16*>(out), lse, sh,
+                                     static_cast<const float*>(nullptr));
     else
-      ga::fwd::attn_fwd_kernel<false><<<grid, ga::fwd::kThreads, ga::fwd::kSmemBytes<false>, s>>>(
-          map_qkv, map_qkv, static_cast<__nv_bfloat16*>(out), lse, sh, nullptr, sched);
+      launch_fwd_kernel<false, false>(sched, grid, n, s, map_qkv, map_qkv,
+                                      static_cast<__nv_bfloat16*>(out), lse, sh,
+                                      static_cast<const float*>(nullptr));
     return (ls = check_launch()) == GA_OK;
   });
   return ls;
@@ -525,11 +552,10 @@ ga_status gpt2_attn_fwd_fp8(const void* qkv8, const float* scales, void* out, fl
   if (!make_map_u8(&map_v, qkv8, inner, T, B, CU_TENSOR_MAP_SWIZZLE_NONE)) return GA_ERR_CUDA;
   const ga::AttnShape sh = make_shape(B, T, H, scale);
   ga_status ls = GA_OK;
-  for_each_fwd_launch(B, T, H, info->num_sms, [&](const ga::fwd::ItemSchedule& sched, int grid) {
-    ga::fwd::attn_fwd_kernel<true><<<grid, ga::fwd::kThreads, ga::fwd::kSmemBytes<true>,
-                                     reinterpret_cast<cudaStream_t>(stream)>>>(
-        map_qk, map_v, static_cast<__nv_bfloat16*>(out), lse, sh,
-        scales + ga::fp8::kDequantOffset, sched);
+  for_each_fwd_launch(B, T, H, info->num_sms, [&](const FwdSchedule& sched, int grid, int n) {
+    launch_fwd_kernel<true, false>(sched, grid, n, reinterpret_cast<cudaStream_t>(stream), map_qk,
+                                   map_v, static_cast<__nv_bfloat16*>(out), lse, sh,
+                                   scales + ga::fp8::kDequantOffset);
     return (ls = check_launch()) == GA_OK;
   });
   return ls;
@@ -878,7 +904,7 @@ int gpt2_attn_fwd_item_schedule(int B, int T, int H, int num_sms, int* launch, i
   const long items = static_cast<long>(B) * H * ((n_qt + 1) / 2);
   if (n < items || items > INT32_MAX) return -GA_ERR_INVALID_ARG;
   int n_launch = 0;
-  for_each_fwd_launch(B, T, H, num_sms, [&](const ga::fwd::ItemSchedule& sched, int grid) {
+  for_each_fwd_launch(B, T, H, num_sms, [&](const FwdSchedule& sched, int grid, int) {
     for (int c = 0; c < grid; ++c)
       for (int t = sched.start[c]; t < sched.start[c + 1]; ++t) {
         const long k = sched.base + static_cast<long>(sched.item[t]);
