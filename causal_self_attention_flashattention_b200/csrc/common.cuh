@@ -60,4 +60,29 @@ __device__ __forceinline__ int snake_item(int r, int grid, int cta) {
   return r * grid + ((r & 1) ? (grid - 1 - cta) : cta);
 }
 
+// A deal of work items to the CTAs of one launch, computed on the host and
+// passed by value (a kernel parameter): CTA c runs items base + item[t] for t
+// in [start[c], start[c + 1]), in that order, at most kSchedSlots of them.
+// Every launch copies the whole parameter, so kernels come with a small and a
+// large table, and the host picks the smaller one that holds the deal.
+constexpr int kSchedMaxCtas = 160;
+constexpr int kSchedSlots = 64;
+template <int kItems>
+struct ItemSchedule {
+  int base;
+  uint16_t start[kSchedMaxCtas + 1];
+  uint16_t item[kItems];
+};
+
+// Copies this CTA's items into items[0 .. n) and n into items[kSchedSlots];
+// every thread of the block takes part, and a barrier must follow before the
+// list is read.
+template <int kItems>
+__device__ __forceinline__ void load_item_list(const ItemSchedule<kItems>& sched, int* items) {
+  const int t0 = sched.start[blockIdx.x];
+  const int n = min(sched.start[blockIdx.x + 1] - t0, kSchedSlots);
+  if (threadIdx.x == 0) items[kSchedSlots] = n;
+  for (int t = threadIdx.x; t < n; t += blockDim.x) items[t] = sched.base + sched.item[t0 + t];
+}
+
 }  // namespace ga

@@ -79,24 +79,12 @@ __device__ __forceinline__ uint32_t col_o(int q) { return 384 + q * 64; }
 template <bool kFp8>
 constexpr int kQKBytes = kFp8 ? kTileBytes / 2 : kTileBytes;
 
-// The deal of items to CTAs for one launch, computed on the host and passed
-// by value (a kernel parameter): CTA c runs items base + item[t] for t in
-// [start[c], start[c + 1]), in that order, at most kSchedSlots of them. The
-// host fills it longest-processing-time first (items in decode_item order,
-// heaviest first, each to the CTA with the least work so far) and splits a
-// forward whose items do not fit one table into several launches. Every
-// launch copies the whole parameter, so a launch of at most kSchedSmall items
-// takes the small table.
-constexpr int kSchedMaxCtas = 160;
+// The forward's item tables (ItemSchedule): the host fills them longest
+// processing time first (items in decode_item order, heaviest first, each to
+// the CTA with the least work so far) and splits a forward whose items do not
+// fit the large one into several launches.
 constexpr int kSchedSmall = 1024;
 constexpr int kSchedMaxItems = 6144;
-constexpr int kSchedSlots = 64;
-template <int kItems>
-struct ItemSchedule {
-  int base;
-  uint16_t start[kSchedMaxCtas + 1];
-  uint16_t item[kItems];
-};
 
 template <bool kFp8>
 struct alignas(1024) Smem {
@@ -200,12 +188,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap map_qkv,
   // This CTA's items, in order, and their count in the last slot (the
   // __syncthreads below publishes them to every role).
   __shared__ int items[kSchedSlots + 1];
-  {
-    const int t0 = sched.start[blockIdx.x];
-    const int n = min(sched.start[blockIdx.x + 1] - t0, kSchedSlots);
-    if (threadIdx.x == 0) items[kSchedSlots] = n;
-    for (int t = threadIdx.x; t < n; t += blockDim.x) items[t] = sched.base + sched.item[t0 + t];
-  }
+  load_item_list(sched, items);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {

@@ -129,7 +129,10 @@ const DeviceInfo* setup_device(int dev) {
 
   if (cudaFuncSetAttribute(ga::bwd::dkdv::attn_bwd_dkdv_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(ga::bwd::dkdv::kSmemBytes)) != cudaSuccess)
+                           static_cast<int>(ga::bwd::dkdv::kSmemBytes)) != cudaSuccess ||
+      cudaFuncSetAttribute(ga::bwd::dq::attn_bwd_dq_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ga::bwd::dq::kSmemBytes)) != cudaSuccess)
     return nullptr;
   if (cudaFuncSetAttribute(ga::bwd::fused::attn_bwd_fused_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -159,10 +162,6 @@ const DeviceInfo* setup_device(int dev) {
       return nullptr;
     info.pair_clusters = n;
   }
-  if (cudaFuncSetAttribute(ga::bwd::dq::attn_bwd_dq_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(ga::bwd::dq::kSmemBytes)) != cudaSuccess)
-    return nullptr;
   info.ready = true;
   return &info;
 }
@@ -330,38 +329,32 @@ ga::AttnShape make_shape(int B, int T, int H, float scale) {
 
 int grid_for(int items, int num_sms) { return items < num_sms ? items : num_sms; }
 
-using FwdSchedule = ga::fwd::ItemSchedule<ga::fwd::kSchedMaxItems>;
-using FwdScheduleSmall = ga::fwd::ItemSchedule<ga::fwd::kSchedSmall>;
+// Item deals (ga::ItemSchedule), longest processing time first. Items come
+// heaviest first (their numbering in the kernel); each goes to the CTA with
+// the least work so far, the lowest index on ties. An item's work is counted
+// in half-tile steps: 2n for its n tiles plus a constant that stands for what
+// an item costs beyond its tiles (the forward's first S product, the previous
+// item's output and the swap of its warpgroups' tiles), chosen by A/B at
+// B=16 T=1024 H=12 among 0, 1.26 and 2.5 tile steps (2.5 was fastest).
+constexpr long kFwdItemCost2 = 5;
 
-// The forward's deal of items to CTAs (ga::fwd::ItemSchedule), longest
-// processing time first. Items come heaviest first (the order of
-// decode_item); each goes to the CTA with the least work so far, the lowest
-// index on ties. An item with n key tiles costs 2n + kItemStartCost2 in
-// half-tile steps: the constant stands for what an item costs beyond its
-// tiles (its first S product, the previous item's output, the swap of the
-// two warpgroups' tiles), about two and a half tile steps when measured
-// (A/B of 0, 1.26 and 2.5 at B=16 T=1024 H=12; 2.5 was fastest).
-constexpr long kItemStartCost2 = 5;
-
-// Deals items [k0, k1) to `grid` CTAs into *s. False if a CTA would get more
-// than kSchedSlots items (the caller then deals fewer items per launch).
-bool build_fwd_schedule(FwdSchedule* s, int n_qt, int bh, long k0, long k1, int grid) {
-  const int n_pairs = (n_qt + 1) / 2;
+// Deals items [k0, k1) to `grid` CTAs into *s; cost(k) is item k's work.
+// False if a CTA would get more than kSchedSlots items (the caller then deals
+// fewer items per launch).
+template <int kItems, class Cost>
+bool build_schedule(ga::ItemSchedule<kItems>* s, long k0, long k1, int grid, Cost cost) {
   const long n = k1 - k0;
-  if (grid <= 0 || grid > ga::fwd::kSchedMaxCtas || n <= 0 || n > ga::fwd::kSchedMaxItems)
-    return false;
+  if (grid <= 0 || grid > ga::kSchedMaxCtas || n <= 0 || n > kItems) return false;
   using Load = std::pair<long, int>;  // (work so far, CTA)
   std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
   for (int c = 0; c < grid; ++c) heap.push(Load(0, c));
   std::vector<int> owner(n), count(grid, 0);
   for (long k = k0; k < k1; ++k) {
-    const int p = n_pairs - 1 - static_cast<int>(k / bh);
-    const int n_kv = (2 * p + 1) < n_qt ? 2 * p + 2 : 2 * p + 1;
     const Load least = heap.top();
     heap.pop();
     owner[k - k0] = least.second;
-    if (++count[least.second] > ga::fwd::kSchedSlots) return false;
-    heap.push(Load(least.first + 2L * n_kv + kItemStartCost2, least.second));
+    if (++count[least.second] > ga::kSchedSlots) return false;
+    heap.push(Load(least.first + cost(k), least.second));
   }
   int off = 0;
   for (int c = 0; c < grid; ++c) {
@@ -375,51 +368,36 @@ bool build_fwd_schedule(FwdSchedule* s, int n_qt, int bh, long k0, long k1, int 
   return true;
 }
 
-// Calls launch(schedule, grid, items) once per launch of a forward over B*H heads
-// and T rows on num_sms SMs, in item order. One launch unless the items do
-// not fit one table. The deal of a one-launch forward is cached per (query
-// tiles, heads, SMs) in a fixed table replaced round-robin under its own
-// mutex. Returns false if a launch failed (launch() returned false).
-struct SchedCacheEntry {
-  bool used = false;
-  int n_qt = 0, bh = 0, num_sms = 0;
-  FwdSchedule sched;
-  int grid = 0;
-  int n = 0;  // items in the launch
+// One-launch deals, cached per (query tiles, heads, SMs) in a fixed table
+// replaced round-robin under its own mutex.
+template <int kItems>
+struct SchedCache {
+  struct Entry {
+    bool used = false;
+    int n_qt = 0, bh = 0, num_sms = 0;
+    ga::ItemSchedule<kItems> sched;
+    int grid = 0;
+    int n = 0;  // items in the launch
+  };
+  static constexpr int kSize = 8;
+  std::mutex mutex;
+  Entry entries[kSize];
+  int next = 0;
 };
-constexpr int kSchedCacheSize = 8;
-std::mutex g_sched_mutex;
-SchedCacheEntry g_sched_cache[kSchedCacheSize];
-int g_sched_next = 0;
+SchedCache<ga::fwd::kSchedMaxItems> g_fwd_sched;
 
-// Launches attn_fwd_kernel<kFp8, kV16> over the n items of `sched` on `grid`
-// CTAs, with the small item table when they fit it.
-template <bool kFp8, bool kV16, class... Args>
-void launch_fwd_kernel(const FwdSchedule& sched, int grid, int n, cudaStream_t stream,
-                       Args... args) {
-  const size_t smem = kFp8 ? ga::fwd::kSmemBytes<true> : ga::fwd::kSmemBytes<false>;
-  if (n <= ga::fwd::kSchedSmall) {
-    FwdScheduleSmall small;
-    small.base = sched.base;
-    std::copy(sched.start, sched.start + grid + 1, small.start);
-    std::copy(sched.item, sched.item + n, small.item);
-    ga::fwd::attn_fwd_kernel<kFp8, kV16, ga::fwd::kSchedSmall>
-        <<<grid, ga::fwd::kThreads, smem, stream>>>(args..., small);
-  } else {
-    ga::fwd::attn_fwd_kernel<kFp8, kV16, ga::fwd::kSchedMaxItems>
-        <<<grid, ga::fwd::kThreads, smem, stream>>>(args..., sched);
-  }
-}
-
-template <class Launch>
-bool for_each_fwd_launch(int B, int T, int H, int num_sms, Launch launch) {
-  const int n_qt = (T + ga::kBlockM - 1) / ga::kBlockM, bh = B * H;
-  const long items = static_cast<long>(bh) * ((n_qt + 1) / 2);
-  FwdSchedule sched;
+// Calls launch(schedule, grid, items) once per launch of a kernel over
+// `items` items of n_qt query tiles and bh heads on num_sms SMs, in item
+// order: one launch unless the items do not fit one table. Returns false if a
+// launch failed (launch() returned false).
+template <int kItems, class Cost, class Launch>
+bool for_each_launch(SchedCache<kItems>& cache, int n_qt, int bh, long items, int num_sms,
+                     Cost cost, Launch launch) {
+  ga::ItemSchedule<kItems> sched;
   int cached_grid = 0, cached_n = 0;
   {
-    std::lock_guard<std::mutex> lock(g_sched_mutex);
-    for (const SchedCacheEntry& e : g_sched_cache)
+    std::lock_guard<std::mutex> lock(cache.mutex);
+    for (const auto& e : cache.entries)
       if (e.used && e.n_qt == n_qt && e.bh == bh && e.num_sms == num_sms) {
         cached_grid = e.grid;
         cached_n = e.n;
@@ -430,19 +408,19 @@ bool for_each_fwd_launch(int B, int T, int H, int num_sms, Launch launch) {
       }
   }
   if (cached_grid > 0) return launch(sched, cached_grid, cached_n);
-  long chunk = ga::fwd::kSchedMaxItems;
+  long chunk = kItems;
   for (long k0 = 0; k0 < items;) {
     const long k1 = std::min(items, k0 + chunk);
     const int grid = static_cast<int>(
-        std::min<long>(k1 - k0, std::min(num_sms, ga::fwd::kSchedMaxCtas)));
-    if (!build_fwd_schedule(&sched, n_qt, bh, k0, k1, grid)) {
+        std::min<long>(k1 - k0, std::min(num_sms, ga::kSchedMaxCtas)));
+    if (!build_schedule(&sched, k0, k1, grid, cost)) {
       chunk /= 2;  // fits at the latest once chunk <= kSchedSlots
       continue;
     }
     if (k0 == 0 && k1 == items) {
-      std::lock_guard<std::mutex> lock(g_sched_mutex);
-      SchedCacheEntry& e = g_sched_cache[g_sched_next];
-      g_sched_next = (g_sched_next + 1) % kSchedCacheSize;
+      std::lock_guard<std::mutex> lock(cache.mutex);
+      auto& e = cache.entries[cache.next];
+      cache.next = (cache.next + 1) % SchedCache<kItems>::kSize;
       e.sched = sched;
       e.grid = grid;
       e.n = static_cast<int>(k1 - k0);
@@ -455,6 +433,79 @@ bool for_each_fwd_launch(int B, int T, int H, int num_sms, Launch launch) {
     k0 = k1;
   }
   return true;
+}
+
+// The forward: item k is a pair of query tiles with n_kv(k) key tiles.
+template <class Launch>
+bool for_each_fwd_launch(int B, int T, int H, int num_sms, Launch launch) {
+  const int n_qt = ga::ceil_div(T, ga::kBlockM), bh = B * H, n_pairs = (n_qt + 1) / 2;
+  auto cost = [=](long k) {
+    const int p = n_pairs - 1 - static_cast<int>(k / bh);
+    const int n_kv = (2 * p + 1) < n_qt ? 2 * p + 2 : 2 * p + 1;
+    return 2L * n_kv + kFwdItemCost2;
+  };
+  return for_each_launch(g_fwd_sched, n_qt, bh, static_cast<long>(bh) * n_pairs, num_sms, cost,
+                         launch);
+}
+
+// Calls fn(table) with the deal of `sched` (n items on grid CTAs) in the
+// smaller table type that holds it: every launch copies its whole parameter.
+template <int kSmall, int kLarge, class Fn>
+void with_table(const ga::ItemSchedule<kLarge>& sched, int grid, int n, Fn fn) {
+  if (n <= kSmall) {
+    ga::ItemSchedule<kSmall> small;
+    small.base = sched.base;
+    std::copy(sched.start, sched.start + grid + 1, small.start);
+    std::copy(sched.item, sched.item + n, small.item);
+    fn(small);
+  } else {
+    fn(sched);
+  }
+}
+
+template <class Table>
+constexpr int table_items() {
+  return static_cast<int>(sizeof(Table::item) / sizeof(Table::item[0]));
+}
+
+// Writes the deal of each launch into launch/cta/pos (indexed by item).
+struct DealWriter {
+  int* launch;
+  int* cta;
+  int* pos;
+  int n_launch = 0;
+  template <class Sched>
+  bool operator()(const Sched& sched, int grid, int) {
+    for (int c = 0; c < grid; ++c)
+      for (int t = sched.start[c]; t < sched.start[c + 1]; ++t) {
+        const long k = sched.base + static_cast<long>(sched.item[t]);
+        launch[k] = n_launch;
+        cta[k] = c;
+        pos[k] = t - sched.start[c];
+      }
+    ++n_launch;
+    return true;
+  }
+};
+
+bool deal_args_ok(int B, int T, int H, int num_sms, const int* launch, const int* cta,
+                  const int* pos) {
+  return launch != nullptr && cta != nullptr && pos != nullptr && B > 0 && T > 0 && H > 0 &&
+         num_sms > 0;
+}
+
+
+// Launches attn_fwd_kernel<kFp8, kV16> over the n items of `sched` on `grid`
+// CTAs.
+template <bool kFp8, bool kV16, class... Args>
+void launch_fwd_kernel(const ga::ItemSchedule<ga::fwd::kSchedMaxItems>& sched, int grid, int n,
+                       cudaStream_t stream, Args... args) {
+  const size_t smem = kFp8 ? ga::fwd::kSmemBytes<true> : ga::fwd::kSmemBytes<false>;
+  with_table<ga::fwd::kSchedSmall>(sched, grid, n, [&](const auto& table) {
+    constexpr int kN = table_items<std::decay_t<decltype(table)>>();
+    ga::fwd::attn_fwd_kernel<kFp8, kV16, kN><<<grid, ga::fwd::kThreads, smem, stream>>>(args...,
+                                                                                        table);
+  });
 }
 
 size_t delta_bytes(int B, int T, int H) {
@@ -487,7 +538,7 @@ ga_status launch_fwd(const void* qkv, void* out, float* lse, int B, int T, int H
   const ga::AttnShape sh = make_shape(B, T, H, scale);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   ga_status ls = GA_OK;
-  for_each_fwd_launch(B, T, H, info->num_sms, [&](const FwdSchedule& sched, int grid, int n) {
+  for_each_fwd_launch(B, T, H, info->num_sms, [&](const auto& sched, int grid, int n) {
     if (v16)
       launch_fwd_kernel<false, true>(sched, grid, n, s, map_qkv, map_qkv,
                                      static_cast<__nv_bfloat16*>(out), lse, sh,
@@ -552,7 +603,7 @@ ga_status gpt2_attn_fwd_fp8(const void* qkv8, const float* scales, void* out, fl
   if (!make_map_u8(&map_v, qkv8, inner, T, B, CU_TENSOR_MAP_SWIZZLE_NONE)) return GA_ERR_CUDA;
   const ga::AttnShape sh = make_shape(B, T, H, scale);
   ga_status ls = GA_OK;
-  for_each_fwd_launch(B, T, H, info->num_sms, [&](const FwdSchedule& sched, int grid, int n) {
+  for_each_fwd_launch(B, T, H, info->num_sms, [&](const auto& sched, int grid, int n) {
     launch_fwd_kernel<true, false>(sched, grid, n, reinterpret_cast<cudaStream_t>(stream), map_qk,
                                    map_v, static_cast<__nv_bfloat16*>(out), lse, sh,
                                    scales + ga::fp8::kDequantOffset);
@@ -897,25 +948,13 @@ int gpt2_attn_version(void) { return 100; }
 
 int gpt2_attn_fwd_item_schedule(int B, int T, int H, int num_sms, int* launch, int* cta,
                                 int* pos, long n) {
-  if (launch == nullptr || cta == nullptr || pos == nullptr || B <= 0 || T <= 0 || H <= 0 ||
-      num_sms <= 0)
-    return -GA_ERR_INVALID_ARG;
-  const int n_qt = (T + ga::kBlockM - 1) / ga::kBlockM;
+  if (!deal_args_ok(B, T, H, num_sms, launch, cta, pos)) return -GA_ERR_INVALID_ARG;
+  const int n_qt = ga::ceil_div(T, ga::kBlockM);
   const long items = static_cast<long>(B) * H * ((n_qt + 1) / 2);
   if (n < items || items > INT32_MAX) return -GA_ERR_INVALID_ARG;
-  int n_launch = 0;
-  for_each_fwd_launch(B, T, H, num_sms, [&](const FwdSchedule& sched, int grid, int) {
-    for (int c = 0; c < grid; ++c)
-      for (int t = sched.start[c]; t < sched.start[c + 1]; ++t) {
-        const long k = sched.base + static_cast<long>(sched.item[t]);
-        launch[k] = n_launch;
-        cta[k] = c;
-        pos[k] = t - sched.start[c];
-      }
-    ++n_launch;
-    return true;
-  });
-  return n_launch;
+  DealWriter w{launch, cta, pos};
+  for_each_fwd_launch(B, T, H, num_sms, [&](const auto& s, int g, int m) { return w(s, g, m); });
+  return w.n_launch;
 }
 
 }  // extern "C"
