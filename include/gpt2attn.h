@@ -79,6 +79,11 @@ typedef enum {
  * than 2^-15). A v entry beyond fp16's range (|v| >= 65536, inf or NaN) is
  * reported as GA_ERR_RANGE by gpt2_attn_last_device_status; the outputs of
  * that call are then undefined.
+ * The work items (one (b,h) and a pair of query tiles each) are dealt to a
+ * persistent grid of at most one CTA per SM by the host, longest processing
+ * time first (gpt2_attn_fwd_item_schedule returns the deal); the deal is
+ * cached per shape. A forward of more than 6144 items is split into several
+ * launches on `stream`. The deal never changes the result.
  */
 ga_status gpt2_attn_fwd(const void* qkv, void* out, float* lse,
                         int B, int T, int H, int D, float scale,
