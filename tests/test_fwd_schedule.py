@@ -126,3 +126,23 @@ def test_split_into_launches_when_the_table_is_full():
 def test_bad_arguments(args):
     with pytest.raises(ValueError):
         ops.fwd_item_schedule(*args)
+
+
+def test_cached_deal_is_the_built_one():
+    """The first call builds and caches the deal; later calls (the cache hit,
+    as every forward after the first takes) return the same one."""
+    first = ops.fwd_item_schedule(5, 896, 7, 148)
+    for _ in range(3):
+        again = ops.fwd_item_schedule(5, 896, 7, 148)
+        assert again[3] == first[3]
+        for a, b in zip(again[:3], first[:3]):
+            assert (a == b).all()
+
+
+def test_more_sms_than_one_table_describes():
+    """On a device with more than 160 SMs a launch uses 160 CTAs."""
+    launch, cta, pos, n = ops.fwd_item_schedule(16, 1024, 12, 200)
+    assert n == 1 and cta.max() == MAX_CTAS - 1
+    nkv = items_of(16, 1024, 12)
+    ld = loads(nkv, cta, MAX_CTAS)
+    assert ld.max() <= ld.sum() / MAX_CTAS + cost2(nkv).max()
